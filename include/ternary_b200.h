@@ -1,0 +1,188 @@
+/*
+ * ternary_b200.h -- C ABI of libternary_b200.so: the ternary-g128 linear layer
+ * with a signed block-Hadamard rotation, on NVIDIA B200 (sm_100a).
+ *
+ * What the layer is (the pages' sections):
+ *   - Ternary g128 weights: each weight t is -1, 0 or +1 and each run of 128
+ *     consecutive weights along K shares one FP16 scale s, so w = s * t
+ *     (news.ditty.ir, "Bonsai 2 27B", second paragraph; ai4coding.ru,
+ *     "What is a ternary model").
+ *   - A signed Hadamard rotation on blocks of 1024 inputs is folded into every
+ *     weight matrix; its inverse must be applied to the activations at run
+ *     time, and forgetting it gives silently wrong output (news.ditty.ir,
+ *     second and third paragraphs; openbonsai.org, "How it works", "Rotate").
+ *   - Multiplying by a ternary weight is an add, a subtract or nothing
+ *     (ai4coding.ru, "What is a ternary model", last paragraph).
+ *   - Two packings are named (a dense trit packing and a 2-bit slot packing,
+ *     news.ditty.ir, paragraph on the CUDA GGUF files); the byte layouts below
+ *     are this library's own.
+ *
+ * Conventions for every entry point:
+ *   - Shapes: W is [N, K] (N outputs, K inputs), x is [M, K], y is [M, N],
+ *     all row-major and densely packed (row stride = row length).
+ *   - Every data pointer is a DEVICE pointer owned by the caller.  The library
+ *     never allocates device memory and keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All device
+ *     work is enqueued asynchronously on it; results are ready when the stream
+ *     says so.
+ *   - Arguments are validated synchronously, before anything is enqueued; a
+ *     non-zero status means nothing was launched (TB_ERR_CUDA excepted, which
+ *     reports a failed launch).
+ *   - Bad data (codes outside {-1,0,1}, invalid packed bytes) is never trapped:
+ *     pack/unpack count it into an optional device uint32 counter (added to,
+ *     never reset, by the call).
+ *   - Calls are thread-safe.  The only library state is a per-device cache of
+ *     device attributes and one per-device fault word (see
+ *     tb_get_device_fault).
+ *
+ * Packed formats (codes only; the FP16 scales always live in a separate
+ * [N, K/128] array, row-major, scale g of row n covering k = 128g..128g+127):
+ *   TB_FMT_2BIT  : c = t + 1 in {0,1,2}.  Byte i of a row holds k = 4i..4i+3,
+ *                  weight k = 4i+j in bits 2j..2j+1.  Row stride K/4 bytes.
+ *                  c = 3 is invalid.  2 + 16/128 = 2.125 bits per weight.
+ *   TB_FMT_BASE3 : each 128-group is its own run of 26 bytes.  Bytes 0..24 hold
+ *                  k = 5i..5i+4 as sum_j c_{5i+j} * 3^j; byte 25 holds
+ *                  k = 125..127 as c125 + 3 c126 + 9 c127 + 108 (digits 3 and 4
+ *                  are the padding value 1).  Row stride 26*K/128 bytes.  A byte
+ *                  >= 243, or a last byte whose digits 3, 4 are not both 1, is
+ *                  invalid.  1.625 + 16/128 = 1.75 bits per weight.
+ *
+ * Rotation (this library's reading of "signed block Hadamard"): for block b of
+ * 1024 inputs with signs d_b in {-1,+1}, R_b = diag(d_b) H / 32 where H is the
+ * Sylvester Hadamard matrix of order 1024 in natural order.  The weights are
+ * stored as W' = W R; the run time applies x' = R^T x, i.e. per block
+ * x'_b = H (d_b * x_b) / 32, so that W' x' = W x.
+ */
+#ifndef TERNARY_B200_H
+#define TERNARY_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int tb_status;
+#define TB_OK 0
+#define TB_ERR_NULL 1      /* a required pointer is NULL                      */
+#define TB_ERR_SHAPE 2     /* a size is <= 0 or breaks a divisibility rule    */
+#define TB_ERR_DTYPE 3     /* unsupported dtype or dtype combination          */
+#define TB_ERR_FORMAT 4    /* unknown packed format                            */
+#define TB_ERR_ALIGN 5     /* a pointer breaks its alignment rule              */
+#define TB_ERR_CUDA 6      /* a CUDA call or launch failed                     */
+#define TB_ERR_WORKSPACE 7 /* workspace NULL or smaller than required          */
+#define TB_ERR_DEVICE 8    /* current device is not a B200-class sm_100 GPU    */
+
+typedef int tb_format;
+#define TB_FMT_2BIT 0
+#define TB_FMT_BASE3 1
+
+typedef int tb_dtype;
+#define TB_BF16 0
+#define TB_FP16 1
+#define TB_FP32 2
+#define TB_INT8 3
+#define TB_INT32 4
+
+typedef int tb_path;
+#define TB_PATH_AUTO 0   /* choose by shape (what tb_ternary_linear does)       */
+#define TB_PATH_GEMV 1   /* CUDA-core streaming kernel (dp4a on 16-bit fixed-point
+                            activations), for M <= 4                           */
+#define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
+                            s*t in shared memory, fp32 accumulators in TMEM)    */
+#define TB_PATH_SIMPLE 3 /* plain per-row kernel: any K % 128, any alignment    */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* tb_status_string(tb_status st);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int tb_version(void);
+
+/* Bytes of packed codes for an [N, K] matrix in format f (scales excluded;
+ * they take N * K/128 * 2 bytes).  Returns 0 for an unknown format, N <= 0,
+ * K <= 0 or K % 128 != 0. */
+size_t tb_packed_bytes(tb_format f, int64_t N, int64_t K);
+
+/* Pack int8 codes [N, K] (values -1, 0, +1) into format f.
+ *   codes  : device, N*K int8.
+ *   packed : device, tb_packed_bytes(f, N, K) bytes, written in full.
+ *   d_invalid_count : device uint32 or NULL.  Every code outside {-1,0,1} is
+ *            packed as 0 and, when non-NULL, adds 1 to *d_invalid_count.
+ * Requires K % 128 == 0; codes and packed 16-byte aligned (else TB_ERR_ALIGN).
+ * Defined by the format description above; no counterpart kernel on the pages. */
+tb_status tb_pack_ternary(tb_format f, const int8_t* codes, int64_t N, int64_t K,
+                          uint8_t* packed, uint32_t* d_invalid_count, void* stream);
+
+/* Unpack format-f bytes into int8 codes [N, K].  Invalid slots/bytes decode to
+ * 0 and, when d_invalid_count is non-NULL, add 1 each (2-bit: per slot holding
+ * 3; base-3: per invalid byte).  Same size/alignment rules as tb_pack_ternary. */
+tb_status tb_unpack_ternary(tb_format f, const uint8_t* packed, int64_t N, int64_t K,
+                            int8_t* codes, uint32_t* d_invalid_count, void* stream);
+
+/* Apply the block rotation to each row of x [M, K] (K % 1024 == 0).
+ *   inverse = 0 : y_b = H (d_b * x_b) / 32   (x' = R^T x, the run-time step
+ *                 before a rotated linear layer, news.ditty.ir third paragraph)
+ *   inverse = 1 : y_b = d_b * (H x_b) / 32   (x = R x')
+ *   xt in {BF16, FP16, FP32}, yt in {BF16, FP16, FP32}; computed in fp32.
+ *   signs : device, K int8, each -1 or +1 (other values are used as given).
+ *   y may equal x when xt == yt (in place); any other overlap is undefined.
+ * Alignment: x, y 16-byte aligned. */
+tb_status tb_hadamard_rotate(const void* x, tb_dtype xt, void* y, tb_dtype yt,
+                             const int8_t* signs, int64_t M, int64_t K, int inverse,
+                             void* stream);
+
+/* Device workspace bytes tb_ternary_linear needs for these sizes (any path,
+ * any dtype).  0 means none.  Returns 0 also for invalid sizes. */
+size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K);
+
+/* y = x' W^T with W the ternary g128 matrix given by (packed, scales, f).
+ *   x       : device [M, K].  xt in {BF16, FP16, FP32}: float mode; xt = INT8:
+ *             integer mode.
+ *   signs   : device [K] int8 or NULL.  Non-NULL: x is unrotated and the
+ *             rotation x' = R^T x is applied first (needs K % 1024 == 0).
+ *             NULL: x is taken as already rotated.  Must be NULL in integer mode.
+ *   scales  : device [N, K/128] fp16 bit patterns.  Ignored in integer mode.
+ *   y       : device [M, N]; yt in {FP32, BF16} in float mode, INT32 in integer
+ *             mode (y[m,n] = sum_k t[n,k] x[m,k], exact).
+ *   workspace : device, at least tb_ternary_linear_workspace(f, M, N, K) bytes,
+ *             16-byte aligned; its contents on entry do not matter and are
+ *             overwritten.  Must not be shared by calls in flight at once.
+ * Requires M >= 1, N >= 1, K % 128 == 0; packed, scales, x, y 16-byte aligned
+ * (else the plain kernel is used; pointers only need natural alignment then).
+ * Float results agree with the exact product to relative L2 error <= 2e-3 and
+ * per element <= 1e-2 * max|s| * ||x_m||_2.  Invalid packed bytes give
+ * unspecified values in the affected outputs (no fault). */
+tb_status tb_ternary_linear(const void* x, tb_dtype xt, const uint8_t* packed,
+                            const uint16_t* scales, tb_format f, int64_t M, int64_t N,
+                            int64_t K, const int8_t* signs, void* y, tb_dtype yt,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* tb_ternary_linear with the kernel path chosen by the caller (tests, tuning).
+ * A path that cannot take the arguments returns TB_ERR_SHAPE without launching
+ * anything: GEMV needs float mode, M <= 4, K % 1024 == 0 and 16-byte aligned
+ * packed/scales; GEMM needs float mode, K % 1024 == 0 and aligned pointers;
+ * SIMPLE takes everything tb_ternary_linear takes. */
+tb_status tb_ternary_linear_ex(const void* x, tb_dtype xt, const uint8_t* packed,
+                               const uint16_t* scales, tb_format f, int64_t M, int64_t N,
+                               int64_t K, const int8_t* signs, void* y, tb_dtype yt,
+                               void* workspace, size_t ws_bytes, tb_path path,
+                               void* stream);
+
+/* Which path tb_ternary_linear would take for these arguments (a tb_path
+ * value), or -1 if it would reject them. */
+int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64_t K,
+                           int has_signs, int aligned16);
+
+/* Read, and with clear != 0 reset, the fault word of the current device.  Every
+ * wait inside the library's kernels is bounded; a wait that gives up (a
+ * producer that never delivered) records a non-zero code here and the kernel
+ * returns early instead of hanging, leaving its outputs incomplete.  0 = no
+ * fault recorded.  Synchronous (waits for the device's work to finish). */
+tb_status tb_get_device_fault(uint32_t* code, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERNARY_B200_H */

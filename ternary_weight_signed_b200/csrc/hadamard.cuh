@@ -1,0 +1,291 @@
+// Signed block-Hadamard rotation of activations (fast Walsh-Hadamard
+// transform on 1024-blocks) and the activation-prep kernels of the linear
+// paths, which fuse the rotation with what each path reads:
+//   * prep_gemv: rotate, then per 128-group 16-bit fixed point split into two
+//     int8 planes (hi, lo) laid out for dp4a against the packed 2-bit words;
+//   * prep_f32 / prep_f16: rotate, then store fp32 (plain kernel) or fp16
+//     (tensor-core kernel).
+//
+// Rotation (news.ditty.ir, Bonsai 2 27B, second and third paragraphs): the
+// weights carry W' = W R, R = blockdiag(diag(d_b) H / 32); the run time applies
+// x'_b = H (d_b * x_b) / 32.  H is the Sylvester matrix in natural order, which
+// is exactly what the in-place radix-2 butterfly below produces.
+//
+// One CTA of 128 threads per (row, 1024-block): each thread holds 8
+// consecutive elements; butterfly distances 1..4 run in registers, 8..128 over
+// warp shuffles, 256 and 512 through shared memory.
+#pragma once
+#include "tb_device.cuh"
+
+namespace tb {
+
+constexpr int kHB = 1024;        // Hadamard block
+constexpr int kHThreads = 128;   // threads per block transform
+constexpr float kHNorm = 0.03125f;  // 1 / sqrt(1024), exact
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float v[8]);
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float v[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load8<__half>(const __half* p, float v[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float v[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store8(T* p, const float v[8]);
+template <>
+__device__ __forceinline__ void store8<float>(float* p, const float v[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <>
+__device__ __forceinline__ void store8<__half>(__half* p, const float v[8]) {
+  uint4 u;
+  __half2* h = reinterpret_cast<__half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const float v[8]) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+// load8 for a pointer of unknown alignment: vector load when 16-byte aligned,
+// element loads otherwise (the plain kernel accepts any naturally aligned x).
+template <typename T>
+__device__ __forceinline__ void load8_any(const T* p, float v[8]) {
+  if ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+    load8<T>(p, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = to_f32<T>(p[i]);
+  }
+}
+
+__device__ __forceinline__ void load_signs8(const int8_t* s, float d[8]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(s);
+  const int8_t* c = reinterpret_cast<const int8_t*>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d[i] = static_cast<float>(c[i]);
+}
+
+// Unnormalised Walsh-Hadamard transform of one 1024-block held as v[8] per
+// thread (thread t owns elements 8t..8t+7).  Result: each thread again owns
+// elements 8t..8t+7 of the transform.  `sm` is 1024 floats of shared memory;
+// all 128 threads must call.
+__device__ __forceinline__ void fwht1024(float v[8], float* sm) {
+  const int t = threadIdx.x;
+  // distances 1, 2, 4: inside the thread
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  }
+  // distances 8 .. 128: partner thread t ^ (h / 8), inside the warp
+#pragma unroll
+  for (int lm = 1; lm < 32; lm <<= 1) {
+    const bool upper = (t & lm) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[i], lm);
+      v[i] = upper ? (o - v[i]) : (v[i] + o);
+    }
+  }
+  // distances 256 and 512: across the 4 warps, through shared memory
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sm[8 * t + i] = v[i];
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int j = t + 128 * r;  // 0..255
+    float a = sm[j], b = sm[j + 256], c = sm[j + 512], d = sm[j + 768];
+    const float a1 = a + b, b1 = a - b, c1 = c + d, d1 = c - d;
+    sm[j] = a1 + c1;
+    sm[j + 512] = a1 - c1;
+    sm[j + 256] = b1 + d1;
+    sm[j + 768] = b1 - d1;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = sm[8 * t + i];
+}
+
+// Loads the thread's 8 elements of block `blk` of row `row`, applies the
+// forward rotation (signs, transform, 1/32) when `signs` is non-null, else
+// only converts to fp32.  All 128 threads must call.
+template <typename TIn>
+__device__ __forceinline__ void load_rotated8(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
+                                              int64_t row, int blk, int64_t K, float v[8],
+                                              float* sm) {
+  const int64_t k0 = static_cast<int64_t>(blk) * kHB + 8 * threadIdx.x;
+  load8_any<TIn>(x + row * K + k0, v);
+  if (signs != nullptr) {
+    float d[8];
+    load_signs8(signs + k0, d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= d[i];
+    fwht1024(v, sm);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= kHNorm;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tb_hadamard_rotate: grid (M, K/1024), 128 threads.
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kHThreads) rotate_kernel(const TIn* x, TOut* y,
+                                                           const int8_t* __restrict__ signs,
+                                                           int64_t K, int inverse) {
+  __shared__ float sm[kHB];
+  const int64_t row = blockIdx.x;
+  const int blk = blockIdx.y;
+  const int64_t k0 = static_cast<int64_t>(blk) * kHB + 8 * threadIdx.x;
+  float v[8], d[8];
+  load8<TIn>(x + row * K + k0, v);
+  load_signs8(signs + k0, d);
+  if (!inverse) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= d[i];
+  }
+  fwht1024(v, sm);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] *= kHNorm;
+  if (inverse) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= d[i];
+  }
+  store8<TOut>(y + row * K + k0, v);
+}
+
+// ---------------------------------------------------------------------------
+// GEMV activation prep.  Per token row, the workspace holds
+//   hi[K] int8 | lo[K] int8 | info[K/32] {float e, int qsum}
+// (2.25 K bytes).  For each 128-group g: e_g = max|x'_g| / 32512,
+// q = rint(x' / e_g) in [-32512, 32512], q = 256 hi + lo with hi in
+// [-127, 127], lo in [-128, 127].  info for quarter-group j (32 codes) holds
+// e of its group and the sum of q over the quarter.
+// Within each 16-code chunk the planes are permuted so that byte 4j + b holds
+// code k = 4b + j: then ((w >> 2j) & 0x03030303) of a packed 2-bit word and
+// activation word j of the chunk line up byte for byte in dp4a.
+constexpr float kQMax = 32512.0f;
+
+__host__ __device__ constexpr int64_t gemv_act_row_bytes(int64_t K) { return 2 * K + K / 4; }
+
+template <typename TIn>
+__global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restrict__ x,
+                                                              const int8_t* __restrict__ signs,
+                                                              uint8_t* __restrict__ ws, int64_t K) {
+  __shared__ float sm[kHB];
+  __shared__ uint2 hi_s[128];
+  __shared__ uint2 lo_s[128];
+  pdl_launch_dependents();
+  const int64_t row = blockIdx.x;
+  const int blk = blockIdx.y;
+  const int t = threadIdx.x;
+  float v[8];
+  load_rotated8<TIn>(x, signs, row, blk, K, v, sm);
+  // group max over 16 threads (128 elements)
+  float mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float e = mx / kQMax;
+  const float inv = mx > 0.f ? kQMax / mx : 0.f;
+  int q[8];
+  int qs = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int qi = __float2int_rn(v[i] * inv);
+    qi = max(-32512, min(32512, qi));
+    q[i] = qi;
+    qs += qi;
+  }
+  qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+  qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+  // Thread pair (2c, 2c+1) holds chunk c; element i of thread half h is code
+  // k = 8h + i = 4b + j with b = 2h + i/4, j = i%4 -> permuted byte 4j + b.
+  __syncthreads();  // sm reuse guard not needed for hi_s/lo_s, keep ordering simple
+  uint8_t* hb = reinterpret_cast<uint8_t*>(hi_s);
+  uint8_t* lb = reinterpret_cast<uint8_t*>(lo_s);
+  const int c = t >> 1, h = t & 1;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int hi = (q[i] + 128) >> 8;
+    const int lo = q[i] - (hi << 8);
+    const int b = 2 * h + (i >> 2), j = i & 3;
+    hb[16 * c + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(hi));
+    lb[16 * c + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(lo));
+  }
+  __syncthreads();
+  uint8_t* base = ws + row * gemv_act_row_bytes(K);
+  const int64_t k0 = static_cast<int64_t>(blk) * kHB;
+  reinterpret_cast<uint2*>(base + k0)[t] = hi_s[t];
+  reinterpret_cast<uint2*>(base + K + k0)[t] = lo_s[t];
+  if ((t & 3) == 0) {
+    int2 inf;
+    inf.x = __float_as_int(e);
+    inf.y = qs;
+    reinterpret_cast<int2*>(base + 2 * K)[(k0 >> 5) + (t >> 2)] = inf;
+  }
+}
+
+// Rotated (or converted) activations in fp32 / fp16 for the plain and the
+// tensor-core kernels: grid (M, K/1024).
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kHThreads) prep_store_kernel(const TIn* __restrict__ x,
+                                                               const int8_t* __restrict__ signs,
+                                                               TOut* __restrict__ out, int64_t K) {
+  __shared__ float sm[kHB];
+  pdl_launch_dependents();
+  const int64_t row = blockIdx.x;
+  const int blk = blockIdx.y;
+  float v[8];
+  load_rotated8<TIn>(x, signs, row, blk, K, v, sm);
+  store8<TOut>(out + row * K + static_cast<int64_t>(blk) * kHB + 8 * threadIdx.x, v);
+}
+
+// Conversion only (no rotation), for K % 1024 != 0: one thread per element.
+template <typename TIn, typename TOut>
+__global__ void convert_kernel(const TIn* __restrict__ x, TOut* __restrict__ out, int64_t n) {
+  pdl_launch_dependents();
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i < n) out[i] = from_f32<TOut>(to_f32<TIn>(x[i]));
+}
+
+}  // namespace tb

@@ -1,0 +1,132 @@
+// Pack / unpack kernels for the two packed formats (byte layouts in
+// include/ternary_b200.h).  Elementwise, memory-bound, one thread per output
+// word (2-bit) or per 128-group (base-3).  Bit-exact by construction; invalid
+// input is counted, never trapped.
+#pragma once
+#include "tb_device.cuh"
+
+namespace tb {
+
+__device__ __forceinline__ void count_invalid(uint32_t bad, uint32_t* counter) {
+  if (counter == nullptr) return;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+  if ((threadIdx.x & 31) == 0 && bad) atomicAdd(counter, bad);
+}
+
+// Biased code c = t + 1 for a valid t, else 1 (t = 0); *bad counts invalids.
+__device__ __forceinline__ uint32_t biased_code(int t, uint32_t* bad) {
+  const bool ok = (t >= -1) && (t <= 1);
+  *bad += ok ? 0u : 1u;
+  return ok ? static_cast<uint32_t>(t + 1) : 1u;
+}
+
+// One thread per 16 codes -> one 32-bit word (4 packed bytes).
+__global__ void pack_2bit_kernel(const int4* __restrict__ codes, uint32_t* __restrict__ out,
+                                 int64_t nwords, uint32_t* counter) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint32_t bad = 0;
+  if (i < nwords) {
+    const int4 v = codes[i];
+    const int8_t* c = reinterpret_cast<const int8_t*>(&v);
+    uint32_t w = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w |= biased_code(c[j], &bad) << (2 * j);
+    out[i] = w;
+  }
+  count_invalid(bad, counter);
+}
+
+__global__ void unpack_2bit_kernel(const uint32_t* __restrict__ in, int4* __restrict__ codes,
+                                   int64_t nwords, uint32_t* counter) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint32_t bad = 0;
+  if (i < nwords) {
+    const uint32_t w = in[i];
+    int4 v;
+    int8_t* c = reinterpret_cast<int8_t*>(&v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t s = (w >> (2 * j)) & 3u;
+      bad += (s == 3u);
+      c[j] = (s == 3u) ? int8_t(0) : static_cast<int8_t>(static_cast<int>(s) - 1);
+    }
+    codes[i] = v;
+  }
+  count_invalid(bad, counter);
+}
+
+// One thread per 128-group: 128 codes in, 26 bytes out (13 16-bit stores; a
+// group starts at an even byte offset).
+__global__ void pack_base3_kernel(const int4* __restrict__ codes, uint16_t* __restrict__ out,
+                                  int64_t ngroups, uint32_t* counter) {
+  const int64_t gi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint32_t bad = 0;
+  if (gi < ngroups) {
+    uint32_t c[130];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int4 v = codes[gi * 8 + q];
+      const int8_t* t = reinterpret_cast<const int8_t*>(&v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) c[16 * q + j] = biased_code(t[j], &bad);
+    }
+    c[128] = 1u;  // padding digits of the last byte
+    c[129] = 1u;
+    uint16_t* o = out + gi * 13;
+#pragma unroll
+    for (int h = 0; h < 13; ++h) {
+      uint32_t b[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const uint32_t* d = c + 5 * (2 * h + e);
+        b[e] = d[0] + 3u * d[1] + 9u * d[2] + 27u * d[3] + 81u * d[4];
+      }
+      o[h] = static_cast<uint16_t>(b[0] | (b[1] << 8));
+    }
+  }
+  count_invalid(bad, counter);
+}
+
+__global__ void unpack_base3_kernel(const uint16_t* __restrict__ in, int4* __restrict__ codes,
+                                    int64_t ngroups, uint32_t* counter) {
+  const int64_t gi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint32_t bad = 0;
+  if (gi < ngroups) {
+    int8_t t[130];
+    const uint16_t* p = in + gi * 13;
+#pragma unroll
+    for (int h = 0; h < 13; ++h) {
+      const uint32_t pair = p[h];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int byte_idx = 2 * h + e;
+        uint32_t v = (pair >> (8 * e)) & 0xffu;
+        uint32_t dig[5];
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+          dig[j] = v % 3u;
+          v /= 3u;
+        }
+        const uint32_t raw = (pair >> (8 * e)) & 0xffu;
+        bool invalid = raw >= 243u;
+        if (byte_idx == 25) invalid = invalid || dig[3] != 1u || dig[4] != 1u;
+        bad += invalid ? 1u : 0u;
+#pragma unroll
+        for (int j = 0; j < 5; ++j)
+          t[5 * byte_idx + j] = invalid ? int8_t(0) : static_cast<int8_t>(static_cast<int>(dig[j]) - 1);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      int4 v;
+      int8_t* o = reinterpret_cast<int8_t*>(&v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) o[j] = t[16 * q + j];
+      codes[gi * 8 + q] = v;
+    }
+  }
+  count_invalid(bad, counter);
+}
+
+}  // namespace tb

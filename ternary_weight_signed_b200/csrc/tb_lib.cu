@@ -1,0 +1,574 @@
+// libternary_b200.so: the C ABI declared in include/ternary_b200.h.
+//
+// One translation unit: the kernels live in the included .cuh files.  Host
+// code here validates arguments (before anything is enqueued), picks a kernel
+// path, builds TMA descriptors and launches on the caller's stream.  Nothing
+// here allocates device memory.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <unordered_set>
+
+#include "ternary_b200.h"
+#include "tb_device.cuh"
+
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "hadamard.cuh"
+#include "pack.cuh"
+#include "simple.cuh"
+
+namespace {
+
+using namespace tb;
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+
+// ------------------------------------------------------------------ device
+struct DevInfo {
+  bool valid = false;
+  int sm_count = 0;
+  int max_smem_optin = 0;
+  int cc_major = 0;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[64];
+std::unordered_set<uint64_t> g_smem_set;  // (function, device) pairs with the attribute set
+
+tb_status current_device(const DevInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.valid) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return TB_ERR_CUDA;
+    }
+    d.sm_count = prop.multiProcessorCount;
+    d.max_smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+    d.cc_major = prop.major;
+    d.valid = true;
+  }
+  if (d.cc_major != 10) return TB_ERR_DEVICE;
+  *out = &d;
+  return TB_OK;
+}
+
+// Raises a kernel's dynamic shared-memory limit to the device maximum, once
+// per (kernel, device).
+template <typename F>
+tb_status allow_smem(F* fn, const DevInfo* d) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t key = reinterpret_cast<uint64_t>(reinterpret_cast<const void*>(fn)) ^
+                       (static_cast<uint64_t>(dev) << 56);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_smem_set.count(key)) return TB_OK;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, d->max_smem_optin) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  g_smem_set.insert(key);
+  return TB_OK;
+}
+
+tb_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TB_OK : TB_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+tb_status get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return TB_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return TB_OK;
+}
+
+// Row-major 2-D tensor [rows, cols] of `dtype` elements, box [box_rows, box_cols].
+tb_status make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int esize, const void* base,
+                      uint64_t cols, uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols,
+                      uint32_t box_rows, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  (void)esize;
+  if (get_encoder() != TB_OK) return TB_ERR_CUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TB_OK : TB_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ helpers
+bool is_float_dtype(int t) { return t == TB_BF16 || t == TB_FP16 || t == TB_FP32; }
+int dtype_size(int t) {
+  switch (t) {
+    case TB_BF16:
+    case TB_FP16: return 2;
+    case TB_FP32:
+    case TB_INT32: return 4;
+    case TB_INT8: return 1;
+    default: return 0;
+  }
+}
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+template <typename Kern, typename... Args>
+tb_status launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  return TB_OK;
+}
+
+// ------------------------------------------------------------------ rotate dispatch
+template <typename TIn, typename TOut>
+void launch_rotate(const void* x, void* y, const int8_t* signs, int64_t M, int64_t K, int inverse,
+                   cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(M), static_cast<unsigned>(K / kHB));
+  rotate_kernel<TIn, TOut><<<grid, kHThreads, 0, st>>>(static_cast<const TIn*>(x),
+                                                       static_cast<TOut*>(y), signs, K, inverse);
+}
+
+template <typename TIn>
+void launch_rotate_out(int yt, const void* x, void* y, const int8_t* signs, int64_t M, int64_t K,
+                       int inverse, cudaStream_t st) {
+  switch (yt) {
+    case TB_BF16: launch_rotate<TIn, __nv_bfloat16>(x, y, signs, M, K, inverse, st); break;
+    case TB_FP16: launch_rotate<TIn, __half>(x, y, signs, M, K, inverse, st); break;
+    default: launch_rotate<TIn, float>(x, y, signs, M, K, inverse, st); break;
+  }
+}
+
+// ------------------------------------------------------------------ linear: validation
+struct LinearArgs {
+  const void* x;
+  int xt;
+  const uint8_t* packed;
+  const uint16_t* scales;
+  int f;
+  int64_t M, N, K;
+  const int8_t* signs;
+  void* y;
+  int yt;
+  void* ws;
+  size_t ws_bytes;
+  cudaStream_t st;
+};
+
+size_t workspace_bytes(int64_t M, int64_t K) {
+  const size_t b = static_cast<size_t>(4) * static_cast<size_t>(M) * static_cast<size_t>(K);
+  return (b + 255) & ~static_cast<size_t>(255);
+}
+
+bool fast_aligned(const LinearArgs& a) {
+  return aligned(a.packed, 16) && aligned(a.scales, 16) && aligned(a.x, 16) && aligned(a.y, 16) &&
+         aligned(a.ws, 16) && (a.signs == nullptr || aligned(a.signs, 16));
+}
+
+int gemv_smem_stages(int64_t M, int64_t K, const DevInfo* d, size_t* smem_out) {
+  const int64_t act = (M * gemv_act_row_bytes(K) + 1023) & ~int64_t(1023);
+  const int64_t avail = static_cast<int64_t>(d->max_smem_optin) - act - 1024;
+  int ns = static_cast<int>(avail / (kStageBytes + 16));
+  if (ns > 8) ns = 8;
+  if (ns < 2) return 0;
+  *smem_out = static_cast<size_t>(act + static_cast<int64_t>(ns) * kStageBytes + (2 * ns + 1) * 8 + 1024);
+  return ns;
+}
+
+bool gemv_ok(const LinearArgs& a) {
+  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGemvMaxM &&
+         a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30);
+}
+
+bool gemm_ok(const LinearArgs& a) {
+  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.K % 1024 == 0 && fast_aligned(a) &&
+         (a.M + kGemmBM - 1) / kGemmBM <= 65535 && a.N < (int64_t(1) << 30);
+}
+
+int auto_path(const LinearArgs& a) {
+  if (a.xt == TB_INT8) return TB_PATH_SIMPLE;
+  if (gemv_ok(a)) return TB_PATH_GEMV;
+  if (gemm_ok(a)) return TB_PATH_GEMM;
+  return TB_PATH_SIMPLE;
+}
+
+// ------------------------------------------------------------------ linear: GEMV
+template <typename TIn>
+tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
+  const int M = static_cast<int>(a.M);
+  uint8_t* act = static_cast<uint8_t*>(a.ws);
+  dim3 pgrid(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
+  prep_gemv_kernel<TIn><<<pgrid, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, act, a.K);
+  if (launch_status() != TB_OK) return TB_ERR_CUDA;
+
+  CUtensorMap tm_w, tm_s;
+  const int64_t G = a.K / 128;
+  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, 64,
+                  kGemvQuadRows) != TB_OK)
+    return TB_ERR_CUDA;
+  if (make_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, a.N, G * 2, 8,
+                  kGemvQuadRows) != TB_OK)
+    return TB_ERR_CUDA;
+  size_t smem = 0;
+  const int ns = gemv_smem_stages(a.M, a.K, d, &smem);
+  if (ns == 0) return TB_ERR_SHAPE;
+  GemvParams p;
+  p.act = act;
+  p.y = a.y;
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.nquads = static_cast<int>((a.N + kGemvQuadRows - 1) / kGemvQuadRows);
+  p.nstages = ns;
+  const int grid = p.nquads < d->sm_count ? p.nquads : d->sm_count;
+#define TB_GEMV_CASE(MM)                                                                        \
+  case MM:                                                                                      \
+    if (a.yt == TB_FP32) {                                                                      \
+      auto k = gemv_2bit_kernel<MM, float>;                                                     \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                        \
+      return launch_pdl(k, dim3(grid), dim3(kGemvThreads), smem, a.st, tm_w, tm_s, p);          \
+    } else {                                                                                    \
+      auto k = gemv_2bit_kernel<MM, __nv_bfloat16>;                                             \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                        \
+      return launch_pdl(k, dim3(grid), dim3(kGemvThreads), smem, a.st, tm_w, tm_s, p);          \
+    }
+  switch (M) {
+    TB_GEMV_CASE(1)
+    TB_GEMV_CASE(2)
+    TB_GEMV_CASE(3)
+    TB_GEMV_CASE(4)
+    default: return TB_ERR_SHAPE;
+  }
+#undef TB_GEMV_CASE
+}
+
+tb_status run_gemv(const LinearArgs& a, const DevInfo* d) {
+  switch (a.xt) {
+    case TB_BF16: return run_gemv_typed<__nv_bfloat16>(a, d);
+    case TB_FP16: return run_gemv_typed<__half>(a, d);
+    default: return run_gemv_typed<float>(a, d);
+  }
+}
+
+// ------------------------------------------------------------------ linear: plain kernel
+template <int FMT>
+tb_status run_simple_fmt(const LinearArgs& a) {
+  const dim3 grid(static_cast<unsigned>((a.N + kSimpleWarps - 1) / kSimpleWarps));
+  const dim3 block(32 * kSimpleWarps);
+  const int M = static_cast<int>(a.M), N = static_cast<int>(a.N), K = static_cast<int>(a.K);
+  const __half* sc = reinterpret_cast<const __half*>(a.scales);
+  if (a.xt == TB_INT8) {
+    simple_linear_kernel<FMT, true, int8_t, int32_t><<<grid, block, 0, a.st>>>(
+        static_cast<const int8_t*>(a.x), a.packed, sc, static_cast<int32_t*>(a.y), M, N, K);
+    return launch_status();
+  }
+  float* xf = static_cast<float*>(a.ws);
+  if (a.signs != nullptr) {
+    const dim3 pg(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
+    switch (a.xt) {
+      case TB_BF16:
+        prep_store_kernel<__nv_bfloat16, float><<<pg, kHThreads, 0, a.st>>>(
+            static_cast<const __nv_bfloat16*>(a.x), a.signs, xf, a.K);
+        break;
+      case TB_FP16:
+        prep_store_kernel<__half, float><<<pg, kHThreads, 0, a.st>>>(static_cast<const __half*>(a.x),
+                                                                      a.signs, xf, a.K);
+        break;
+      default:
+        prep_store_kernel<float, float><<<pg, kHThreads, 0, a.st>>>(static_cast<const float*>(a.x),
+                                                                     a.signs, xf, a.K);
+        break;
+    }
+  } else {
+    const int64_t n = a.M * a.K;
+    const unsigned g = static_cast<unsigned>((n + 255) / 256);
+    switch (a.xt) {
+      case TB_BF16:
+        convert_kernel<__nv_bfloat16, float><<<g, 256, 0, a.st>>>(static_cast<const __nv_bfloat16*>(a.x),
+                                                                  xf, n);
+        break;
+      case TB_FP16:
+        convert_kernel<__half, float><<<g, 256, 0, a.st>>>(static_cast<const __half*>(a.x), xf, n);
+        break;
+      default:
+        convert_kernel<float, float><<<g, 256, 0, a.st>>>(static_cast<const float*>(a.x), xf, n);
+        break;
+    }
+  }
+  if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  if (a.yt == TB_FP32)
+    return launch_pdl(simple_linear_kernel<FMT, false, float, float>, grid, block, 0, a.st,
+                      static_cast<const float*>(xf), a.packed, sc, static_cast<float*>(a.y), M, N, K);
+  return launch_pdl(simple_linear_kernel<FMT, false, float, __nv_bfloat16>, grid, block, 0, a.st,
+                    static_cast<const float*>(xf), a.packed, sc, static_cast<__nv_bfloat16*>(a.y), M,
+                    N, K);
+}
+
+tb_status run_simple(const LinearArgs& a) {
+  return a.f == TB_FMT_2BIT ? run_simple_fmt<0>(a) : run_simple_fmt<1>(a);
+}
+
+// ------------------------------------------------------------------ linear: tensor-core kernel
+template <typename TIn>
+void launch_prep_gemm(const LinearArgs& a, __half* xh) {
+  const dim3 pg(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
+  prep_gemm_kernel<TIn><<<pg, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, xh, a.K);
+}
+
+tb_status run_gemm(const LinearArgs& a, const DevInfo* d) {
+  __half* xh = static_cast<__half*>(a.ws);
+  switch (a.xt) {
+    case TB_BF16: launch_prep_gemm<__nv_bfloat16>(a, xh); break;
+    case TB_FP16: launch_prep_gemm<__half>(a, xh); break;
+    default: launch_prep_gemm<float>(a, xh); break;
+  }
+  if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  CUtensorMap tm_x, tm_w;
+  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGemmBK, kGemmBM,
+                  CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+    return TB_ERR_CUDA;
+  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, kGemmBK / 16,
+                  kGemmBN) != TB_OK)
+    return TB_ERR_CUDA;
+  GemmParams gp;
+  gp.M = static_cast<int>(a.M);
+  gp.N = static_cast<int>(a.N);
+  gp.K = static_cast<int>(a.K);
+  gp.y = a.y;
+  gp.scales = a.scales;
+  const dim3 grid(static_cast<unsigned>((a.N + kGemmBN - 1) / kGemmBN),
+                  static_cast<unsigned>((a.M + kGemmBM - 1) / kGemmBM));
+  if (a.yt == TB_FP32) {
+    auto k = gemm_2bit_tc_kernel<float>;
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
+    return launch_pdl(k, grid, dim3(kGemmThreads), kGemmSmemBytes, a.st, tm_x, tm_w, gp);
+  }
+  auto k = gemm_2bit_tc_kernel<__nv_bfloat16>;
+  if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
+  return launch_pdl(k, grid, dim3(kGemmThreads), kGemmSmemBytes, a.st, tm_x, tm_w, gp);
+}
+
+tb_status validate_linear(const LinearArgs& a) {
+  if (a.f != TB_FMT_2BIT && a.f != TB_FMT_BASE3) return TB_ERR_FORMAT;
+  const bool int_mode = a.xt == TB_INT8;
+  if (a.x == nullptr || a.packed == nullptr || a.y == nullptr) return TB_ERR_NULL;
+  if (!int_mode && a.scales == nullptr) return TB_ERR_NULL;
+  if (a.M < 1 || a.N < 1 || a.K < 128 || a.K % 128 != 0) return TB_ERR_SHAPE;
+  if (a.M > kMaxDim || a.N > kMaxDim || a.K > kMaxDim) return TB_ERR_SHAPE;
+  if (a.M * a.K > (int64_t(1) << 40) || a.N * a.K > (int64_t(1) << 44)) return TB_ERR_SHAPE;
+  if (int_mode) {
+    if (a.yt != TB_INT32) return TB_ERR_DTYPE;
+    if (a.signs != nullptr) return TB_ERR_DTYPE;
+  } else {
+    if (!is_float_dtype(a.xt)) return TB_ERR_DTYPE;
+    if (a.yt != TB_FP32 && a.yt != TB_BF16) return TB_ERR_DTYPE;
+    if (a.signs != nullptr && a.K % 1024 != 0) return TB_ERR_SHAPE;
+  }
+  if (!aligned(a.x, dtype_size(a.xt)) || !aligned(a.y, dtype_size(a.yt)) ||
+      (!int_mode && !aligned(a.scales, 2)))
+    return TB_ERR_ALIGN;
+  if (a.signs != nullptr && !aligned(a.signs, 8)) return TB_ERR_ALIGN;
+  if (a.f == TB_FMT_BASE3 && !aligned(a.packed, 2)) return TB_ERR_ALIGN;
+  if (!int_mode) {
+    if (a.ws == nullptr || a.ws_bytes < workspace_bytes(a.M, a.K)) return TB_ERR_WORKSPACE;
+    if (!aligned(a.ws, 16)) return TB_ERR_ALIGN;
+  }
+  return TB_OK;
+}
+
+tb_status linear_impl(const LinearArgs& a, int path) {
+  tb_status st = validate_linear(a);
+  if (st != TB_OK) return st;
+  if (path == TB_PATH_AUTO) path = auto_path(a);
+  if (path == TB_PATH_GEMV && !gemv_ok(a)) return TB_ERR_SHAPE;
+  if (path == TB_PATH_GEMM && !gemm_ok(a)) return TB_ERR_SHAPE;
+  if (path != TB_PATH_GEMV && path != TB_PATH_GEMM && path != TB_PATH_SIMPLE) return TB_ERR_SHAPE;
+  const DevInfo* d = nullptr;
+  st = current_device(&d);
+  if (st != TB_OK) return st;
+  switch (path) {
+    case TB_PATH_GEMV: return run_gemv(a, d);
+    case TB_PATH_GEMM: return run_gemm(a, d);
+    default: return run_simple(a);
+  }
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* tb_status_string(tb_status st) {
+  switch (st) {
+    case TB_OK: return "ok";
+    case TB_ERR_NULL: return "null pointer";
+    case TB_ERR_SHAPE: return "bad shape";
+    case TB_ERR_DTYPE: return "bad dtype";
+    case TB_ERR_FORMAT: return "bad format";
+    case TB_ERR_ALIGN: return "bad alignment";
+    case TB_ERR_CUDA: return "cuda error";
+    case TB_ERR_WORKSPACE: return "workspace missing or too small";
+    case TB_ERR_DEVICE: return "device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+int tb_version(void) { return kVersion; }
+
+size_t tb_packed_bytes(tb_format f, int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0 || K % 128 != 0) return 0;
+  if (f == TB_FMT_2BIT) return static_cast<size_t>(N) * static_cast<size_t>(K / 4);
+  if (f == TB_FMT_BASE3) return static_cast<size_t>(N) * static_cast<size_t>(K / 128) * 26;
+  return 0;
+}
+
+tb_status tb_pack_ternary(tb_format f, const int8_t* codes, int64_t N, int64_t K, uint8_t* packed,
+                          uint32_t* d_invalid_count, void* stream) {
+  if (f != TB_FMT_2BIT && f != TB_FMT_BASE3) return TB_ERR_FORMAT;
+  if (codes == nullptr || packed == nullptr) return TB_ERR_NULL;
+  if (N <= 0 || K <= 0 || K % 128 != 0 || N > kMaxDim || K > kMaxDim) return TB_ERR_SHAPE;
+  if (!aligned(codes, 16) || !aligned(packed, 16) ||
+      (d_invalid_count != nullptr && !aligned(d_invalid_count, 4)))
+    return TB_ERR_ALIGN;
+  const DevInfo* d = nullptr;
+  const tb_status st = current_device(&d);
+  if (st != TB_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  if (f == TB_FMT_2BIT) {
+    const int64_t nw = N * K / 16;
+    pack_2bit_kernel<<<static_cast<unsigned>((nw + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const int4*>(codes), reinterpret_cast<uint32_t*>(packed), nw, d_invalid_count);
+  } else {
+    const int64_t ng = N * K / 128;
+    pack_base3_kernel<<<static_cast<unsigned>((ng + 127) / 128), 128, 0, s>>>(
+        reinterpret_cast<const int4*>(codes), reinterpret_cast<uint16_t*>(packed), ng, d_invalid_count);
+  }
+  return launch_status();
+}
+
+tb_status tb_unpack_ternary(tb_format f, const uint8_t* packed, int64_t N, int64_t K, int8_t* codes,
+                            uint32_t* d_invalid_count, void* stream) {
+  if (f != TB_FMT_2BIT && f != TB_FMT_BASE3) return TB_ERR_FORMAT;
+  if (codes == nullptr || packed == nullptr) return TB_ERR_NULL;
+  if (N <= 0 || K <= 0 || K % 128 != 0 || N > kMaxDim || K > kMaxDim) return TB_ERR_SHAPE;
+  if (!aligned(codes, 16) || !aligned(packed, 16) ||
+      (d_invalid_count != nullptr && !aligned(d_invalid_count, 4)))
+    return TB_ERR_ALIGN;
+  const DevInfo* d = nullptr;
+  const tb_status st = current_device(&d);
+  if (st != TB_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  if (f == TB_FMT_2BIT) {
+    const int64_t nw = N * K / 16;
+    unpack_2bit_kernel<<<static_cast<unsigned>((nw + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const uint32_t*>(packed), reinterpret_cast<int4*>(codes), nw, d_invalid_count);
+  } else {
+    const int64_t ng = N * K / 128;
+    unpack_base3_kernel<<<static_cast<unsigned>((ng + 127) / 128), 128, 0, s>>>(
+        reinterpret_cast<const uint16_t*>(packed), reinterpret_cast<int4*>(codes), ng, d_invalid_count);
+  }
+  return launch_status();
+}
+
+tb_status tb_hadamard_rotate(const void* x, tb_dtype xt, void* y, tb_dtype yt, const int8_t* signs,
+                             int64_t M, int64_t K, int inverse, void* stream) {
+  if (x == nullptr || y == nullptr || signs == nullptr) return TB_ERR_NULL;
+  if (!is_float_dtype(xt) || !is_float_dtype(yt)) return TB_ERR_DTYPE;
+  if (M < 1 || K < 1024 || K % 1024 != 0 || M > kMaxDim || K / 1024 > 65535) return TB_ERR_SHAPE;
+  if (x == y && xt != yt) return TB_ERR_DTYPE;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(signs, 8)) return TB_ERR_ALIGN;
+  const DevInfo* d = nullptr;
+  const tb_status st = current_device(&d);
+  if (st != TB_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  switch (xt) {
+    case TB_BF16: launch_rotate_out<__nv_bfloat16>(yt, x, y, signs, M, K, inverse != 0, s); break;
+    case TB_FP16: launch_rotate_out<__half>(yt, x, y, signs, M, K, inverse != 0, s); break;
+    default: launch_rotate_out<float>(yt, x, y, signs, M, K, inverse != 0, s); break;
+  }
+  return launch_status();
+}
+
+size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K) {
+  if ((f != TB_FMT_2BIT && f != TB_FMT_BASE3) || M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
+  return workspace_bytes(M, K);
+}
+
+tb_status tb_ternary_linear_ex(const void* x, tb_dtype xt, const uint8_t* packed, const uint16_t* scales,
+                               tb_format f, int64_t M, int64_t N, int64_t K, const int8_t* signs,
+                               void* y, tb_dtype yt, void* workspace, size_t ws_bytes, tb_path path,
+                               void* stream) {
+  LinearArgs a{x, xt, packed, scales, f, M, N, K, signs, y, yt, workspace, ws_bytes, as_stream(stream)};
+  return linear_impl(a, path);
+}
+
+tb_status tb_ternary_linear(const void* x, tb_dtype xt, const uint8_t* packed, const uint16_t* scales,
+                            tb_format f, int64_t M, int64_t N, int64_t K, const int8_t* signs, void* y,
+                            tb_dtype yt, void* workspace, size_t ws_bytes, void* stream) {
+  return tb_ternary_linear_ex(x, xt, packed, scales, f, M, N, K, signs, y, yt, workspace, ws_bytes,
+                              TB_PATH_AUTO, stream);
+}
+
+int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64_t K, int has_signs,
+                           int aligned16) {
+  // A stand-in argument set with the requested alignment decides the path.
+  const uintptr_t base = aligned16 ? 0x1000 : 0x1004;
+  LinearArgs a{reinterpret_cast<const void*>(base), xt, reinterpret_cast<const uint8_t*>(base),
+               reinterpret_cast<const uint16_t*>(base), f, M, N, K,
+               has_signs ? reinterpret_cast<const int8_t*>(0x2000) : nullptr,
+               reinterpret_cast<void*>(0x3000), xt == TB_INT8 ? TB_INT32 : TB_FP32,
+               reinterpret_cast<void*>(0x4000), workspace_bytes(M > 0 ? M : 1, K > 0 ? K : 128),
+               nullptr};
+  if (validate_linear(a) != TB_OK) return -1;
+  return auto_path(a);
+}
+
+tb_status tb_get_device_fault(uint32_t* code, int clear) {
+  if (code == nullptr) return TB_ERR_NULL;
+  if (cudaMemcpyFromSymbol(code, tb::g_fault, sizeof(uint32_t)) != cudaSuccess) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  if (clear) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(tb::g_fault, &zero, sizeof(uint32_t)) != cudaSuccess) {
+      cudaGetLastError();
+      return TB_ERR_CUDA;
+    }
+  }
+  return TB_OK;
+}
+
+}  // extern "C"
