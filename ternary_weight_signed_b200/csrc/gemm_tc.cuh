@@ -8,18 +8,23 @@
 //   B = fp16(s * t), which is exact because t is -1, 0 or +1 and s is an fp16
 //       value, so no per-group rescaling of the accumulator is needed.
 //
-// Tile: 128 tokens (TMEM lanes) x 256 weight rows (TMEM columns), K in stages
-// of 64 (one 128-byte swizzle atom of fp16).  Warp roles:
+// Tile: 256 tokens x 256 weight rows, K in stages of 64 (one 128-byte swizzle
+// atom of fp16).  The 256 tokens are two M=128 MMAs that share the unpacked B
+// tile, each with its own 128 x 256 fp32 accumulator (all 512 TMEM columns).
+// Warp roles:
 //   warp 0    : TMA producer (x' tile with 128B swizzle, packed 2-bit codes);
 //   warp 1    : TMEM allocation and the single thread issuing tcgen05.mma;
-//   warps 2-5 : unpack the codes of the stage into fp16 s*t, written straight
-//               into the UMMA K-major 128B-swizzled layout, then the epilogue
-//               (tcgen05.ld of the accumulator, convert, store).
+//   warps 2-9 : unpack the codes of the stage into fp16 s*t (one weight row
+//               per thread), written straight into the UMMA K-major
+//               128B-swizzled layout, then the epilogue (tcgen05.ld of the
+//               accumulators, convert, store).
 //
-// Unpacking: the 2-bit word of 16 codes gives codes j and j+8 in the two
-// halves of ((w >> 2j) & 0x00030003); OR-ing 0x6400 makes the fp16 values
-// 1024 + c exactly, one subtraction gives c, and one fma gives s*c - s = s*t
-// (exact).  That pairs k = j with k = j+8 in each half2, so the prep kernel
+// Unpacking: the 2-bit word of 16 codes holds codes j and j+8 at bits 2j and
+// 2j+16.  For j < 4, ((w >> 2j) & 0x00030003) | 0x64006400 is the fp16 pair
+// (1024 + c_j, 1024 + c_{j+8}); for j >= 4 the same shifted word with mask
+// 0x03000300 gives 1024 + 256 c.  One fma (v - 1024 or v/256 - 4) gives c
+// exactly and one more gives s*c - s = s*t (exact).  That pairs k = j with
+// k = j+8 in each half2, so the prep kernel
 // stores x' with the same order inside every 16-element chunk
 // (k = 0, 8, 1, 9, ..., 7, 15); the contraction over k does not depend on the
 // order as long as both operands share it.
@@ -32,13 +37,15 @@
 
 namespace tb {
 
-constexpr int kGemmBM = 128;
+constexpr int kGemmBM = 256;      // tokens per tile: two MMAs of M = 128
+constexpr int kGemmUM = 128;      // M of one MMA (TMEM lanes)
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 4;
-constexpr int kGemmUnpackWarps = 4;
+constexpr int kGemmStages = 3;
+constexpr int kGemmUnpackWarps = 8;
 constexpr int kGemmThreads = 32 * (2 + kGemmUnpackWarps);
-constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 16 KB
+constexpr int kGemmTmemCols = 512;
+constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 32 KB
 constexpr int kGemmBBytes = kGemmBN * kGemmBK * 2;  // 32 KB
 constexpr int kGemmWBytes = kGemmBN * kGemmBK / 4;  // 4 KB of packed codes
 constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes + kGemmWBytes;
@@ -48,7 +55,7 @@ constexpr int kGemmSmemBytes = kGemmStages * kGemmStageBytes + 1024 /*align*/ + 
 // (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
 // M >> 4 at bits 24-28.
 constexpr uint32_t kGemmIdesc =
-    (1u << 4) | (static_cast<uint32_t>(kGemmBN >> 3) << 17) | (static_cast<uint32_t>(kGemmBM >> 4) << 24);
+    (1u << 4) | (static_cast<uint32_t>(kGemmBN >> 3) << 17) | (static_cast<uint32_t>(kGemmUM >> 4) << 24);
 
 // Shared-memory matrix descriptor for a K-major operand in the canonical
 // 128-byte swizzled layout: rows of 128 bytes, 8-row groups 1024 bytes apart
@@ -210,7 +217,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kGemmBN);
+    tmem_alloc(tmem_slot, kGemmTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -248,24 +255,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t a = smem_u32(smem + s * kGemmStageBytes);
         const uint32_t b = a + kGemmABytes;
 #pragma unroll
-        for (int kk = 0; kk < kGemmBK / 16; ++kk)
-          umma_f16(tmem, umma_desc_sw128(a + 32 * kk), umma_desc_sw128(b + 32 * kk), kGemmIdesc,
-                   (kb | kk) != 0 ? 1u : 0u);
+        for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+          const uint64_t bd = umma_desc_sw128(b + 32 * kk);
+          const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+          umma_f16(tmem, umma_desc_sw128(a + 32 * kk), bd, kGemmIdesc, acc);
+          umma_f16(tmem + kGemmBN, umma_desc_sw128(a + kGemmUM * 128 + 32 * kk), bd, kGemmIdesc, acc);
+        }
         umma_commit(&empty[s]);
       }
       umma_commit(accum);
     }
   } else {
     // ---------------------------------------------------------------- unpack
-    const int ut = threadIdx.x - 64;  // 0..127
+    const int r = threadIdx.x - 64;  // weight row of the tile this thread unpacks (0..255)
     const int G = p.K / 128;
-    __half s_next[2], s_cur[2];
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int n = n0 + ut + 128 * rr;
-      s_next[rr] = __ushort_as_half(n < p.N ? p.scales[static_cast<int64_t>(n) * G] : uint16_t(0));
-      s_cur[rr] = s_next[rr];
-    }
+    const int n = n0 + r;
+    const bool row_ok = n < p.N;
+    const uint16_t* srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
+    __half s_next = __ushort_as_half(row_ok ? srow[0] : uint16_t(0));
+    __half s_cur = s_next;
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
+    const __half2 k1024 = __float2half2_rn(1024.f);
+    const __half2 k1 = __float2half2_rn(1.f);
+    const __half2 kinv256 = __float2half2_rn(1.f / 256.f);
+    const __half2 km4 = __float2half2_rn(-4.f);
     bool ok = true;
     for (int kb = 0; kb < nk && ok; ++kb) {
       const int s = kb % kGemmStages;
@@ -275,40 +288,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if ((kb & 1) == 0) {  // a new 128-group starts: take its scale, prefetch the next
         const int g = kb >> 1;
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          s_cur[rr] = s_next[rr];
-          const int n = n0 + ut + 128 * rr;
-          if (g + 1 < G)
-            s_next[rr] = __ushort_as_half(n < p.N ? p.scales[static_cast<int64_t>(n) * G + g + 1] : uint16_t(0));
-        }
+        s_cur = s_next;
+        if (g + 1 < G) s_next = __ushort_as_half(row_ok ? srow[g + 1] : uint16_t(0));
       }
       uint8_t* st = smem + s * kGemmStageBytes;
-      const uint8_t* wsrc = st + kGemmABytes + kGemmBBytes;
-      uint8_t* bdst = st + kGemmABytes;
-      const __half2 k1024 = __float2half2_rn(1024.f);
+      const uint4 w4 = *reinterpret_cast<const uint4*>(st + kGemmABytes + kGemmBBytes + r * 16);
+      const __half2 s2 = __halves2half2(s_cur, s_cur);
+      const __half2 ns2 = __hneg2(s2);
+      uint8_t* row = st + kGemmABytes + r * 128;
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int r = ut + 128 * rr;
-        const uint4 w4 = *reinterpret_cast<const uint4*>(wsrc + r * 16);
-        const __half2 s2 = __halves2half2(s_cur[rr], s_cur[rr]);
-        const __half2 ns2 = __hneg2(s2);
-        uint8_t* row = bdst + r * 128;
-        const uint32_t sw = static_cast<uint32_t>(r & 7);
+      for (int wd = 0; wd < 4; ++wd) {
+        const uint32_t w = (&w4.x)[wd];
+        uint32_t o[8];
 #pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          const uint32_t w = (&w4.x)[wd];
-          uint32_t o[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t bits = ((w >> (2 * j)) & 0x00030003u) | 0x64006400u;
-            const __half2 c2 = __hsub2(*reinterpret_cast<const __half2*>(&bits), k1024);
-            const __half2 v = __hfma2(c2, s2, ns2);
-            o[j] = *reinterpret_cast<const uint32_t*>(&v);
-          }
-          *reinterpret_cast<uint4*>(row + 16 * ((2 * wd) ^ sw)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(row + 16 * ((2 * wd + 1) ^ sw)) = make_uint4(o[4], o[5], o[6], o[7]);
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t ws = w >> (2 * j);
+          const uint32_t lo = (ws & 0x00030003u) | 0x64006400u;  // 1024 + c_j, 1024 + c_{j+8}
+          const uint32_t hi = (ws & 0x03000300u) | 0x64006400u;  // 1024 + 256 c_{j+4}, ...
+          const __half2 clo = __hfma2(*reinterpret_cast<const __half2*>(&lo), k1, __hneg2(k1024));
+          const __half2 chi = __hfma2(*reinterpret_cast<const __half2*>(&hi), kinv256, km4);
+          const __half2 vlo = __hfma2(clo, s2, ns2);
+          const __half2 vhi = __hfma2(chi, s2, ns2);
+          o[j] = *reinterpret_cast<const uint32_t*>(&vlo);
+          o[j + 4] = *reinterpret_cast<const uint32_t*>(&vhi);
         }
+        *reinterpret_cast<uint4*>(row + 16 * ((2 * wd) ^ sw)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(row + 16 * ((2 * wd + 1) ^ sw)) = make_uint4(o[4], o[5], o[6], o[7]);
       }
       fence_proxy_async_shared();  // generic-proxy stores -> visible to the tensor core
       __syncwarp();
@@ -317,19 +322,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------------- epilogue
     if (mbar_wait(accum, 0, FAULT_WAIT_EPILOGUE)) {
       tc_fence_after();
-      const int q = warp & 3;  // TMEM lane quarter this warp may access
-      const int m = m0 + 32 * q + lane;
+      const int q = warp & 3;             // TMEM lane quarter this warp may access
+      const int h = (warp - 2) >> 2;      // which of the two accumulators
+      const int m = m0 + kGemmUM * h + 32 * q + lane;
       TOut* y = reinterpret_cast<TOut*>(p.y);
       const bool vec = (p.N % static_cast<int>(16 / sizeof(TOut))) == 0;  // 16-byte row alignment
 #pragma unroll 1
       for (int c = 0; c < kGemmBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(32 * c), r);
+        uint32_t v32[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(kGemmBN * h + 32 * c), v32);
         tmem_ld_wait();
         const int nb = n0 + 32 * c;
         if (m < p.M && nb < p.N) {
           const int valid = min(32, p.N - nb);
-          store_row32<TOut>(y + static_cast<int64_t>(m) * p.N + nb, r, valid, vec);
+          store_row32<TOut>(y + static_cast<int64_t>(m) * p.N + nb, v32, valid, vec);
         }
       }
     }
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kGemmBN);
+    tmem_dealloc(tmem, kGemmTmemCols);
   }
 }
 

@@ -198,19 +198,42 @@ bool fast_aligned(const LinearArgs& a) {
          aligned(a.ws, 16) && (a.signs == nullptr || aligned(a.signs, 16));
 }
 
-int gemv_smem_stages(int64_t M, int64_t K, const DevInfo* d, size_t* smem_out) {
-  const int64_t act = (M * gemv_act_row_bytes(K) + 1023) & ~int64_t(1023);
-  const int64_t avail = static_cast<int64_t>(d->max_smem_optin) - act - 1024;
-  int ns = static_cast<int>(avail / (kStageBytes + 16));
-  if (ns > 8) ns = 8;
-  if (ns < 2) return 0;
-  *smem_out = static_cast<size_t>(act + static_cast<int64_t>(ns) * kStageBytes + (2 * ns + 1) * 8 + 1024);
-  return ns;
+struct GemvPlan {
+  int grid, max_rows, seg_rows, nslots;
+  size_t smem;
+};
+
+// Geometry of the decode kernel for these sizes on a device with `sm_count`
+// SMs and `max_smem` bytes of shared memory per block; false if it does not fit.
+bool gemv_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, GemvPlan* out) {
+  if (M < 1 || M > kGemvMaxM || K % 1024 != 0 || N < 1) return false;
+  GemvPlan pl;
+  pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
+  pl.max_rows = static_cast<int>((N + pl.grid - 1) / pl.grid);
+  const int64_t rb = K / 4;
+  int64_t sr = 4 * (kSegBytes / (4 * rb));
+  if (sr < 4) sr = 4;
+  pl.seg_rows = static_cast<int>(sr);
+  const int64_t fixed = gemv_smem_bytes(static_cast<int>(M), K, pl.max_rows, pl.seg_rows, 0) + 8 * 2 * kGemvMaxSlots;
+  int64_t ns = (static_cast<int64_t>(max_smem) - fixed) / (sr * rb);
+  if (ns > kGemvMaxSlots) ns = kGemvMaxSlots;
+  if (ns < kGemvMinSlots) return false;
+  // the activations + scales arrive on one barrier whose byte count is < 2^20
+  if (M * gemv_act_row_bytes(K) + static_cast<int64_t>(pl.max_rows) * (K / 64) >= (int64_t(1) << 20)) return false;
+  pl.nslots = static_cast<int>(ns);
+  pl.smem = static_cast<size_t>(gemv_smem_bytes(static_cast<int>(M), K, pl.max_rows, pl.seg_rows, pl.nslots));
+  *out = pl;
+  return true;
 }
 
+constexpr int kB200Sms = 148;
+constexpr int kB200SmemOptin = 232448;
+
 bool gemv_ok(const LinearArgs& a) {
+  GemvPlan pl;
   return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGemvMaxM &&
-         a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30);
+         a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30) &&
+         gemv_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
 }
 
 bool gemm_ok(const LinearArgs& a) {
@@ -228,43 +251,34 @@ int auto_path(const LinearArgs& a) {
 // ------------------------------------------------------------------ linear: GEMV
 template <typename TIn>
 tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
-  const int M = static_cast<int>(a.M);
+  GemvPlan pl;
+  if (!gemv_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
   uint8_t* act = static_cast<uint8_t*>(a.ws);
   dim3 pgrid(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
   prep_gemv_kernel<TIn><<<pgrid, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, act, a.K);
   if (launch_status() != TB_OK) return TB_ERR_CUDA;
-
-  CUtensorMap tm_w, tm_s;
-  const int64_t G = a.K / 128;
-  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, 64,
-                  kGemvQuadRows) != TB_OK)
-    return TB_ERR_CUDA;
-  if (make_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, a.N, G * 2, 8,
-                  kGemvQuadRows) != TB_OK)
-    return TB_ERR_CUDA;
-  size_t smem = 0;
-  const int ns = gemv_smem_stages(a.M, a.K, d, &smem);
-  if (ns == 0) return TB_ERR_SHAPE;
   GemvParams p;
   p.act = act;
+  p.packed = a.packed;
+  p.scales = a.scales;
   p.y = a.y;
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
-  p.nquads = static_cast<int>((a.N + kGemvQuadRows - 1) / kGemvQuadRows);
-  p.nstages = ns;
-  const int grid = p.nquads < d->sm_count ? p.nquads : d->sm_count;
-#define TB_GEMV_CASE(MM)                                                                        \
-  case MM:                                                                                      \
-    if (a.yt == TB_FP32) {                                                                      \
-      auto k = gemv_2bit_kernel<MM, float>;                                                     \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                        \
-      return launch_pdl(k, dim3(grid), dim3(kGemvThreads), smem, a.st, tm_w, tm_s, p);          \
-    } else {                                                                                    \
-      auto k = gemv_2bit_kernel<MM, __nv_bfloat16>;                                             \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                        \
-      return launch_pdl(k, dim3(grid), dim3(kGemvThreads), smem, a.st, tm_w, tm_s, p);          \
+  p.seg_rows = pl.seg_rows;
+  p.nslots = pl.nslots;
+  p.max_rows = pl.max_rows;
+#define TB_GEMV_CASE(MM)                                                                 \
+  case MM:                                                                               \
+    if (a.yt == TB_FP32) {                                                               \
+      auto k = gemv_2bit_kernel<MM, float>;                                              \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                 \
+      return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, p);         \
+    } else {                                                                             \
+      auto k = gemv_2bit_kernel<MM, __nv_bfloat16>;                                      \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                 \
+      return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, p);         \
     }
-  switch (M) {
+  switch (static_cast<int>(a.M)) {
     TB_GEMV_CASE(1)
     TB_GEMV_CASE(2)
     TB_GEMV_CASE(3)
