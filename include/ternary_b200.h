@@ -174,6 +174,35 @@ tb_status tb_ternary_linear_ex(const void* x, tb_dtype xt, const uint8_t* packed
 int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64_t K,
                            int has_signs, int aligned16);
 
+/* Bytes of the library's fixed device scratch used by tb_ternary_linear_noalloc
+ * (576 KiB: 4 token rows at K = 65536). */
+#define TB_NOALLOC_SCRATCH_BYTES 589824
+
+/* tb_ternary_linear without a workspace argument: the decode (GEMV) path with
+ * its activation scratch in a fixed array inside the library instead of in
+ * caller memory.  The pages have no counterpart; it exists for callers that
+ * cannot allocate device memory: a plugin inside a host runtime that owns every
+ * device allocation and hands plugins none, or a latency-critical decode loop
+ * that must not call cudaMalloc / cudaFree, which can synchronise the device.
+ * It allocates nothing itself (no cudaMalloc, no cudaFree, no library routine
+ * that allocates).
+ *   Takes the arguments of tb_ternary_linear minus the workspace, with the
+ *   GEMV path's rules: float mode, TB_FMT_2BIT, M <= 4, K % 1024 == 0, all
+ *   pointers 16-byte aligned (else TB_ERR_SHAPE / TB_ERR_ALIGN / TB_ERR_DTYPE).
+ *   M * (2K + K/4) bytes of scratch must fit TB_NOALLOC_SCRATCH_BYTES, else
+ *   TB_ERR_WORKSPACE ("too big for the library's fixed scratch") and nothing
+ *   is launched.
+ *   Every GPU that loads the library holds the scratch until the process exits.
+ *   The first call on a device looks up the scratch's device address (a host
+ *   call that does not allocate); make that first call before any stream
+ *   capture.  All calls on a device share the one scratch and every call
+ *   overwrites the part it reads, so nothing needs clearing between calls, but
+ *   calls that can overlap on the GPU (different streams without ordering)
+ *   race on it: order them on one stream. */
+tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* packed,
+                                    const uint16_t* scales, int64_t M, int64_t N, int64_t K,
+                                    const int8_t* signs, void* y, tb_dtype yt, void* stream);
+
 /* Read, and with clear != 0 reset, the fault word of the current device.  Every
  * wait inside the library's kernels is bounded; a wait that gives up (a
  * producer that never delivered) records a non-zero code here and the kernel

@@ -38,6 +38,8 @@ _SIGNATURES = {
                                     _vp, _sz, _int, _vp]),
     "tb_ternary_linear_path": (_int, [_int, _int, _i64, _i64, _i64, _int, _int]),
     "tb_get_device_fault": (_int, [ctypes.POINTER(ctypes.c_uint32), _int]),
+    "tb_ternary_linear_noalloc": (_int, [_vp, _int, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _int,
+                                         _vp]),
 }
 
 _LIB = None
@@ -159,6 +161,18 @@ def tb_ternary_linear_ex(x, xt, packed, scales, fmt, m, n, k, signs, y, yt, work
 
 def tb_ternary_linear_path(xt, fmt, m, n, k, has_signs=True, aligned16=True) -> int:
     return load().tb_ternary_linear_path(xt, _fmt(fmt), m, n, k, int(has_signs), int(aligned16))
+
+
+TB_NOALLOC_SCRATCH_BYTES = 589824
+
+
+def tb_ternary_linear_noalloc(x, xt, packed, scales, m, n, k, signs, y, yt, stream=None,
+                              check=True):
+    """The decode path with the library's fixed scratch instead of a workspace
+    (for callers that cannot allocate device memory; see the C header)."""
+    st = load().tb_ternary_linear_noalloc(_ptr(x), xt, _ptr(packed), _ptr(scales), m, n, k,
+                                          _ptr(signs), _ptr(y), yt, _stream(stream))
+    return _done(st, "tb_ternary_linear_noalloc", check)
 
 
 def tb_get_device_fault(clear=False) -> int:

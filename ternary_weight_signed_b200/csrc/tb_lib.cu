@@ -569,6 +569,62 @@ int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64
   return auto_path(a);
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for callers that cannot allocate (tb_ternary_linear_noalloc).
+// In host code g_noalloc_scratch is only a host-side stand-in for the device
+// array: the kernels get its device address from cudaGetSymbolAddress, looked
+// up once per device with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[TB_NOALLOC_SCRATCH_BYTES];
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[64] = {};
+
+static tb_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return TB_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return TB_OK;
+}
+
+tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* packed,
+                                    const uint16_t* scales, int64_t M, int64_t N, int64_t K,
+                                    const int8_t* signs, void* y, tb_dtype yt, void* stream) {
+  // Validate as tb_ternary_linear would with an ample aligned workspace, then
+  // check the fixed scratch's limit and the GEMV path's own rules.
+  LinearArgs a{x, xt, packed, scales, TB_FMT_2BIT, M, N, K, signs, y, yt,
+               reinterpret_cast<void*>(static_cast<uintptr_t>(256)), workspace_bytes(M > 0 ? M : 1, K > 0 ? K : 128),
+               as_stream(stream)};
+  tb_status st = validate_linear(a);
+  if (st != TB_OK) return st;
+  if (xt == TB_INT8) return TB_ERR_DTYPE;
+  if (M > kGemvMaxM || K % 1024 != 0) return TB_ERR_SHAPE;
+  if (M * gemv_act_row_bytes(K) > static_cast<int64_t>(TB_NOALLOC_SCRATCH_BYTES)) return TB_ERR_WORKSPACE;
+  if (!aligned(packed, 16) || !aligned(scales, 16) || !aligned(x, 16) || !aligned(y, 16) ||
+      (signs != nullptr && !aligned(signs, 16)))
+    return TB_ERR_ALIGN;
+  const DevInfo* d = nullptr;
+  st = current_device(&d);
+  if (st != TB_OK) return st;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != TB_OK) return st;
+  a.ws = scratch;
+  a.ws_bytes = TB_NOALLOC_SCRATCH_BYTES;
+  if (!gemv_ok(a)) return TB_ERR_SHAPE;
+  return run_gemv(a, d);
+}
+
 tb_status tb_get_device_fault(uint32_t* code, int clear) {
   if (code == nullptr) return TB_ERR_NULL;
   if (cudaMemcpyFromSymbol(code, tb::g_fault, sizeof(uint32_t)) != cudaSuccess) {
