@@ -88,10 +88,16 @@ typedef int tb_dtype;
 typedef int tb_path;
 #define TB_PATH_AUTO 0   /* choose by shape (what tb_ternary_linear does)       */
 #define TB_PATH_GEMV 1   /* CUDA-core streaming kernel (dp4a on 16-bit fixed-point
-                            activations), for M <= 4                           */
+                            activations), for M <= 4; for M * K/1024 <= 16 the
+                            rotation runs inside it (one launch per call)       */
 #define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
                             s*t in shared memory, fp32 accumulators in TMEM)    */
 #define TB_PATH_SIMPLE 3 /* plain per-row kernel: any K % 128, any alignment    */
+#define TB_PATH_GEMV_TC 4 /* tcgen05 decode kernel (codes unpacked into TMEM as
+                            the u8 A operand, int8 activation planes as B in
+                            shared memory), for M <= 4 and N <= 148 * 128; same
+                            other rules as TB_PATH_GEMV, slower than it on B200,
+                            never chosen by TB_PATH_AUTO                         */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* tb_status_string(tb_status st);
@@ -175,7 +181,7 @@ int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64
                            int has_signs, int aligned16);
 
 /* Bytes of the library's fixed device scratch used by tb_ternary_linear_noalloc
- * (576 KiB: 4 token rows at K = 65536). */
+ * (576 KiB). */
 #define TB_NOALLOC_SCRATCH_BYTES 589824
 
 /* tb_ternary_linear without a workspace argument: the decode (GEMV) path with
@@ -189,9 +195,10 @@ int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64
  *   Takes the arguments of tb_ternary_linear minus the workspace, with the
  *   GEMV path's rules: float mode, TB_FMT_2BIT, M <= 4, K % 1024 == 0, all
  *   pointers 16-byte aligned (else TB_ERR_SHAPE / TB_ERR_ALIGN / TB_ERR_DTYPE).
- *   M * (2K + K/4) bytes of scratch must fit TB_NOALLOC_SCRATCH_BYTES, else
- *   TB_ERR_WORKSPACE ("too big for the library's fixed scratch") and nothing
- *   is launched.
+ *   The decode path needs max(M * (2K + K/16), 16K + M * K/16) bytes of
+ *   scratch, which must fit TB_NOALLOC_SCRATCH_BYTES (576 KiB: e.g. K <= 32768
+ *   at any M <= 4); larger sizes return TB_ERR_WORKSPACE ("too big for the
+ *   library's fixed scratch") and nothing is launched.
  *   Every GPU that loads the library holds the scratch until the process exits.
  *   The first call on a device looks up the scratch's device address (a host
  *   call that does not allocate); make that first call before any stream

@@ -99,11 +99,12 @@ __device__ __forceinline__ void load_signs8(const int8_t* s, float d[8]) {
 }
 
 // Unnormalised Walsh-Hadamard transform of one 1024-block held as v[8] per
-// thread (thread t owns elements 8t..8t+7).  Result: each thread again owns
-// elements 8t..8t+7 of the transform.  `sm` is 1024 floats of shared memory;
-// all 128 threads must call.
-__device__ __forceinline__ void fwht1024(float v[8], float* sm) {
-  const int t = threadIdx.x;
+// thread (thread t owns elements 8t..8t+7) by a group of 128 threads.  Result:
+// each thread again owns elements 8t..8t+7 of the transform.  `t` is the
+// thread's index in the group (0..127), `bar` a named barrier id private to the
+// group (0 when the group is the whole 128-thread block), `sm` 1024 floats of
+// shared memory private to the group, free for reuse on return.
+__device__ __forceinline__ void fwht1024_group(float v[8], float* sm, int t, int bar) {
   // distances 1, 2, 4: inside the thread
 #pragma unroll
   for (int h = 1; h < 8; h <<= 1) {
@@ -129,21 +130,25 @@ __device__ __forceinline__ void fwht1024(float v[8], float* sm) {
   // distances 256 and 512: across the 4 warps, through shared memory
 #pragma unroll
   for (int i = 0; i < 8; ++i) sm[8 * t + i] = v[i];
-  __syncthreads();
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    const int j = t + 128 * r;  // 0..255
-    float a = sm[j], b = sm[j + 256], c = sm[j + 512], d = sm[j + 768];
+    const int j = t + 128 * r;
+    const float a = sm[j], b = sm[j + 256], c = sm[j + 512], d = sm[j + 768];
     const float a1 = a + b, b1 = a - b, c1 = c + d, d1 = c - d;
     sm[j] = a1 + c1;
     sm[j + 512] = a1 - c1;
     sm[j + 256] = b1 + d1;
     sm[j + 768] = b1 - d1;
   }
-  __syncthreads();
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = sm[8 * t + i];
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");  // sm may be reused after this
 }
+
+// fwht1024_group over a whole 128-thread block.
+__device__ __forceinline__ void fwht1024(float v[8], float* sm) { fwht1024_group(v, sm, threadIdx.x, 0); }
 
 // Loads the thread's 8 elements of block `blk` of row `row`, applies the
 // forward rotation (signs, transform, 1/32) when `signs` is non-null, else
@@ -194,17 +199,19 @@ __global__ void __launch_bounds__(kHThreads) rotate_kernel(const TIn* x, TOut* y
 
 // ---------------------------------------------------------------------------
 // GEMV activation prep.  Per token row, the workspace holds
-//   hi[K] int8 | lo[K] int8 | info[K/32] {float e, int qsum}
-// (2.25 K bytes).  For each 128-group g: e_g = max|x'_g| / 32512,
+//   hi[K] int8 | lo[K] int8 | info[K/128] {float e, int qsum}
+// (2 K + K/16 bytes).  For each 128-group g: e_g = max|x'_g| / 32512,
 // q = rint(x' / e_g) in [-32512, 32512], q = 256 hi + lo with hi in
-// [-127, 127], lo in [-128, 127].  info for quarter-group j (32 codes) holds
-// e of its group and the sum of q over the quarter.
-// Within each 16-code chunk the planes are permuted so that byte 4j + b holds
+// [-127, 127], lo in [-128, 127]; info holds e_g and the sum of q over the group.
+// Within each 16-code word the planes are permuted so that byte 4j + b holds
 // code k = 4b + j: then ((w >> 2j) & 0x03030303) of a packed 2-bit word and
-// activation word j of the chunk line up byte for byte in dp4a.
+// activation word j line up byte for byte in dp4a.  Within each 1024-code
+// block the 16-byte words are stored word-major ([word wd][group g]): word wd
+// of group g sits at 128 wd + 16 g, so the 8 lanes that read word wd of the 8
+// groups of a block touch 128 contiguous bytes (no shared-memory bank conflict).
 constexpr float kQMax = 32512.0f;
 
-__host__ __device__ constexpr int64_t gemv_act_row_bytes(int64_t K) { return 2 * K + K / 4; }
+__host__ __device__ constexpr int64_t gemv_act_row_bytes(int64_t K) { return 2 * K + K / 16; }
 
 template <typename TIn>
 __global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restrict__ x,
@@ -236,32 +243,35 @@ __global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restr
     q[i] = qi;
     qs += qi;
   }
-  qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+  qs += __shfl_xor_sync(0xffffffffu, qs, 1);  // over the group's 16 threads
   qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+  qs += __shfl_xor_sync(0xffffffffu, qs, 4);
+  qs += __shfl_xor_sync(0xffffffffu, qs, 8);
   // Thread pair (2c, 2c+1) holds chunk c; element i of thread half h is code
   // k = 8h + i = 4b + j with b = 2h + i/4, j = i%4 -> permuted byte 4j + b.
   __syncthreads();  // sm reuse guard not needed for hi_s/lo_s, keep ordering simple
   uint8_t* hb = reinterpret_cast<uint8_t*>(hi_s);
   uint8_t* lb = reinterpret_cast<uint8_t*>(lo_s);
-  const int c = t >> 1, h = t & 1;
+  const int c = t >> 1, h = t & 1;           // 16-code word c of the block
+  const int wbase = 128 * (c & 7) + 16 * (c >> 3);  // word (c & 7) of group (c >> 3)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int hi = (q[i] + 128) >> 8;
     const int lo = q[i] - (hi << 8);
     const int b = 2 * h + (i >> 2), j = i & 3;
-    hb[16 * c + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(hi));
-    lb[16 * c + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(lo));
+    hb[wbase + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(hi));
+    lb[wbase + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(lo));
   }
   __syncthreads();
   uint8_t* base = ws + row * gemv_act_row_bytes(K);
   const int64_t k0 = static_cast<int64_t>(blk) * kHB;
   reinterpret_cast<uint2*>(base + k0)[t] = hi_s[t];
   reinterpret_cast<uint2*>(base + K + k0)[t] = lo_s[t];
-  if ((t & 3) == 0) {
+  if ((t & 15) == 0) {
     int2 inf;
     inf.x = __float_as_int(e);
     inf.y = qs;
-    reinterpret_cast<int2*>(base + 2 * K)[(k0 >> 5) + (t >> 2)] = inf;
+    reinterpret_cast<int2*>(base + 2 * K)[(k0 >> 7) + (t >> 4)] = inf;
   }
 }
 

@@ -6,6 +6,7 @@
 // here allocates device memory.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 #include <unordered_set>
 
@@ -14,6 +15,7 @@
 
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_tc.cuh"
 #include "hadamard.cuh"
 #include "pack.cuh"
 #include "simple.cuh"
@@ -189,7 +191,9 @@ struct LinearArgs {
 };
 
 size_t workspace_bytes(int64_t M, int64_t K) {
-  const size_t b = static_cast<size_t>(4) * static_cast<size_t>(M) * static_cast<size_t>(K);
+  size_t b = static_cast<size_t>(4) * static_cast<size_t>(M) * static_cast<size_t>(K);
+  const size_t g = static_cast<size_t>(gtc_ws_bytes(M, K));  // tensor-core decode activations
+  if (g > b) b = g;
   return (b + 255) & ~static_cast<size_t>(255);
 }
 
@@ -211,8 +215,9 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, Gemv
   pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
   pl.max_rows = static_cast<int>((N + pl.grid - 1) / pl.grid);
   const int64_t rb = K / 4;
-  int64_t sr = 4 * (kSegBytes / (4 * rb));
-  if (sr < 4) sr = 4;
+  const int64_t ir = M <= 2 ? 8 : 4;  // rows per work item (see gemv_2bit_kernel)
+  int64_t sr = ir * (kSegBytes / (ir * rb));
+  if (sr < ir) sr = ir;
   pl.seg_rows = static_cast<int>(sr);
   const int64_t fixed = gemv_smem_bytes(static_cast<int>(M), K, pl.max_rows, pl.seg_rows, 0) + 8 * 2 * kGemvMaxSlots;
   int64_t ns = (static_cast<int64_t>(max_smem) - fixed) / (sr * rb);
@@ -226,6 +231,52 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, Gemv
   return true;
 }
 
+struct GtcPlan {
+  int grid, box_rows, rows_box, parts, gpp, nb, nstages, depth;
+  uint32_t w_box_bytes, box_stride, part_bytes, stage_bytes, tmem_cols;
+  size_t smem;
+};
+
+// Geometry of the tensor-core decode kernel; false if these sizes do not fit it.
+bool gtc_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, GtcPlan* out) {
+  if (M < 1 || M > kGtcMaxM || K % 1024 != 0 || N < 1) return false;
+  GtcPlan pl;
+  pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
+  pl.box_rows = static_cast<int>((N + pl.grid - 1) / pl.grid);
+  if (pl.box_rows > 128) return false;
+  pl.rows_box = 32 * ((pl.box_rows + 31) / 32);
+  const int G = static_cast<int>(K / 128);
+  int parts = 128 / pl.rows_box;
+  if (parts > 3) parts = 3;  // TMEM: depth x (32 parts + 16) columns with depth >= 4
+  if (parts > G / 4) parts = G / 4;
+  if (parts < 1) parts = 1;
+  pl.gpp = 4 * ((G + 4 * parts - 1) / (4 * parts));
+  pl.parts = (G + pl.gpp - 1) / pl.gpp;
+  pl.depth = 8;  // a multiple of the 4 step groups
+  if (pl.depth * (32 * pl.parts + 16) > 512) pl.depth = 4;
+  const int cols = pl.depth * (32 * pl.parts + 16);
+  if (cols > 512) return false;
+  pl.tmem_cols = 32;
+  while (static_cast<int>(pl.tmem_cols) < cols) pl.tmem_cols <<= 1;
+  pl.w_box_bytes = static_cast<uint32_t>(pl.box_rows) * 128u;
+  pl.box_stride = (pl.w_box_bytes + 1023u) & ~1023u;
+  for (pl.nb = 2; pl.nb >= 1; --pl.nb) {
+    pl.part_bytes = pl.nb * pl.box_stride + 4u * pl.nb * kGtcAtomBytes;
+    pl.stage_bytes = static_cast<uint32_t>(pl.parts) * pl.part_bytes;
+    const int64_t fixed = gtc_smem_bytes(static_cast<int>(M), K, pl.box_rows, 0, 0, pl.depth) + 8 * 2 * 6;
+    int64_t ns = (static_cast<int64_t>(max_smem) - fixed) / pl.stage_bytes;
+    if (ns > 6) ns = 6;
+    if (ns >= 2) {
+      pl.nstages = static_cast<int>(ns);
+      pl.smem = static_cast<size_t>(
+          gtc_smem_bytes(static_cast<int>(M), K, pl.box_rows, pl.stage_bytes, pl.nstages, pl.depth));
+      *out = pl;
+      return true;
+    }
+  }
+  return false;
+}
+
 constexpr int kB200Sms = 148;
 constexpr int kB200SmemOptin = 232448;
 
@@ -234,6 +285,13 @@ bool gemv_ok(const LinearArgs& a) {
   return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGemvMaxM &&
          a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30) &&
          gemv_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
+}
+
+bool gemv_tc_ok(const LinearArgs& a) {
+  GtcPlan pl;
+  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGemvMaxM &&
+         a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30) &&
+         gtc_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
 }
 
 bool gemm_ok(const LinearArgs& a) {
@@ -249,16 +307,37 @@ int auto_path(const LinearArgs& a) {
 }
 
 // ------------------------------------------------------------------ linear: GEMV
+// The fused kernel has no prep kernel before it to overlap with; launching it
+// without programmatic serialization keeps it ordered after all prior work.
+template <int M>
+tb_status launch_gemv(const LinearArgs& a, const DevInfo* d, const GemvPlan& pl, const GemvParams& p,
+                      bool fused) {
+  auto k = a.yt == TB_FP32 ? gemv_2bit_kernel<M, float> : gemv_2bit_kernel<M, __nv_bfloat16>;
+  if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
+  if (fused) {
+    k<<<dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st>>>(p);
+    return launch_status();
+  }
+  return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, p);
+}
+
 template <typename TIn>
 tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
   GemvPlan pl;
   if (!gemv_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
   uint8_t* act = static_cast<uint8_t*>(a.ws);
-  dim3 pgrid(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
-  prep_gemv_kernel<TIn><<<pgrid, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, act, a.K);
-  if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  const bool fused = a.M * (a.K / kHB) <= kGemvFusedMaxBlocks;
+  if (!fused) {
+    dim3 pgrid(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
+    prep_gemv_kernel<TIn><<<pgrid, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, act, a.K);
+    if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  }
   GemvParams p;
   p.act = act;
+  p.x = a.x;
+  p.signs = a.signs;
+  p.xt = a.xt == TB_BF16 ? 0 : (a.xt == TB_FP16 ? 1 : 2);
+  p.fused = fused ? 1 : 0;
   p.packed = a.packed;
   p.scales = a.scales;
   p.y = a.y;
@@ -267,25 +346,75 @@ tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
   p.seg_rows = pl.seg_rows;
   p.nslots = pl.nslots;
   p.max_rows = pl.max_rows;
-#define TB_GEMV_CASE(MM)                                                                 \
-  case MM:                                                                               \
-    if (a.yt == TB_FP32) {                                                               \
-      auto k = gemv_2bit_kernel<MM, float>;                                              \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                 \
-      return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, p);         \
-    } else {                                                                             \
-      auto k = gemv_2bit_kernel<MM, __nv_bfloat16>;                                      \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                 \
-      return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, p);         \
-    }
   switch (static_cast<int>(a.M)) {
-    TB_GEMV_CASE(1)
-    TB_GEMV_CASE(2)
-    TB_GEMV_CASE(3)
-    TB_GEMV_CASE(4)
+    case 1: return launch_gemv<1>(a, d, pl, p, fused);
+    case 2: return launch_gemv<2>(a, d, pl, p, fused);
+    case 3: return launch_gemv<3>(a, d, pl, p, fused);
+    case 4: return launch_gemv<4>(a, d, pl, p, fused);
     default: return TB_ERR_SHAPE;
   }
-#undef TB_GEMV_CASE
+}
+
+template <typename TIn>
+tb_status run_gemv_tc_typed(const LinearArgs& a, const DevInfo* d, const GtcPlan& pl) {
+  uint8_t* act = static_cast<uint8_t*>(a.ws);
+  const dim3 pgrid(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
+  prep_gemv_tc_kernel<TIn><<<pgrid, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, act, a.K,
+                                                          static_cast<int>(a.M));
+  if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  CUtensorMap tm_w;
+  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, 32,
+                  static_cast<uint32_t>(pl.box_rows), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+    return TB_ERR_CUDA;
+  GemvTcParams p;
+  p.act = act;
+  p.scales = a.scales;
+  p.y = a.y;
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.box_rows = pl.box_rows;
+  p.rows_box = pl.rows_box;
+  p.parts = pl.parts;
+  p.gpp = pl.gpp;
+  p.nb = pl.nb;
+  p.nstages = pl.nstages;
+  p.depth = pl.depth;
+  p.depth_log2 = pl.depth == 8 ? 3 : 2;
+  p.gps_log2 = pl.nb == 2 ? 3 : 2;
+  p.w_box_bytes = pl.w_box_bytes;
+  p.box_stride = pl.box_stride;
+  p.part_bytes = pl.part_bytes;
+  p.stage_bytes = pl.stage_bytes;
+  p.tmem_cols = pl.tmem_cols;
+#define TB_GTC_CASE(MM)                                                                \
+  case MM:                                                                             \
+    if (a.yt == TB_FP32) {                                                             \
+      auto k = gemv_tc_kernel<MM, float>;                                              \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                               \
+      return launch_pdl(k, dim3(pl.grid), dim3(kGtcThreads), pl.smem, a.st, tm_w, p);  \
+    } else {                                                                           \
+      auto k = gemv_tc_kernel<MM, __nv_bfloat16>;                                      \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                               \
+      return launch_pdl(k, dim3(pl.grid), dim3(kGtcThreads), pl.smem, a.st, tm_w, p);  \
+    }
+  switch (static_cast<int>(a.M)) {
+    TB_GTC_CASE(1)
+    TB_GTC_CASE(2)
+    TB_GTC_CASE(3)
+    TB_GTC_CASE(4)
+    default: return TB_ERR_SHAPE;
+  }
+#undef TB_GTC_CASE
+}
+
+tb_status run_gemv_tc(const LinearArgs& a, const DevInfo* d) {
+  GtcPlan pl;
+  if (!gtc_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
+  switch (a.xt) {
+    case TB_BF16: return run_gemv_tc_typed<__nv_bfloat16>(a, d, pl);
+    case TB_FP16: return run_gemv_tc_typed<__half>(a, d, pl);
+    default: return run_gemv_tc_typed<float>(a, d, pl);
+  }
 }
 
 tb_status run_gemv(const LinearArgs& a, const DevInfo* d) {
@@ -428,13 +557,16 @@ tb_status linear_impl(const LinearArgs& a, int path) {
   if (path == TB_PATH_AUTO) path = auto_path(a);
   if (path == TB_PATH_GEMV && !gemv_ok(a)) return TB_ERR_SHAPE;
   if (path == TB_PATH_GEMM && !gemm_ok(a)) return TB_ERR_SHAPE;
-  if (path != TB_PATH_GEMV && path != TB_PATH_GEMM && path != TB_PATH_SIMPLE) return TB_ERR_SHAPE;
+  if (path == TB_PATH_GEMV_TC && !gemv_tc_ok(a)) return TB_ERR_SHAPE;
+  if (path != TB_PATH_GEMV && path != TB_PATH_GEMM && path != TB_PATH_SIMPLE && path != TB_PATH_GEMV_TC)
+    return TB_ERR_SHAPE;
   const DevInfo* d = nullptr;
   st = current_device(&d);
   if (st != TB_OK) return st;
   switch (path) {
     case TB_PATH_GEMV: return run_gemv(a, d);
     case TB_PATH_GEMM: return run_gemm(a, d);
+    case TB_PATH_GEMV_TC: return run_gemv_tc(a, d);
     default: return run_simple(a);
   }
 }
@@ -609,7 +741,8 @@ tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* p
   if (st != TB_OK) return st;
   if (xt == TB_INT8) return TB_ERR_DTYPE;
   if (M > kGemvMaxM || K % 1024 != 0) return TB_ERR_SHAPE;
-  if (M * gemv_act_row_bytes(K) > static_cast<int64_t>(TB_NOALLOC_SCRATCH_BYTES)) return TB_ERR_WORKSPACE;
+  const int64_t need = std::max<int64_t>(M * gemv_act_row_bytes(K), gtc_ws_bytes(M, K));
+  if (need > static_cast<int64_t>(TB_NOALLOC_SCRATCH_BYTES)) return TB_ERR_WORKSPACE;
   if (!aligned(packed, 16) || !aligned(scales, 16) || !aligned(x, 16) || !aligned(y, 16) ||
       (signs != nullptr && !aligned(signs, 16)))
     return TB_ERR_ALIGN;

@@ -246,3 +246,25 @@ def test_gemm_invalid_bytes_no_fault():
     y = prob.linear(GEMM, packed=torch.full_like(prob.packed, 0xFF))
     assert y.shape == (5, 256)
     assert tb.tb_get_device_fault() == 0
+
+
+GEMV_TC = tb.TB_PATH_GEMV_TC
+
+
+@pytest.mark.parametrize("case", WORKLOAD_CASES, ids=lambda c: f"m{c[1]}n{c[2]}k{c[3]}")
+def test_gemv_tensor_core_2bit(case):
+    prob, ref = _problem(case[0], case[1], case[2], case[3], case[4], "2bit", case[5], case[6])
+    _check(prob.linear(GEMV_TC), ref, prob.p)
+
+
+def test_gemv_tensor_core_rejects_rows_beyond_tmem():
+    """More rows than 148 CTAs x 128 TMEM lanes: the tensor-core decode kernel
+    refuses the shape; the CUDA-core kernel takes it."""
+    prob, ref = _problem(24, 2, 20480, 1024, 0.33, "2bit")
+    ws_bytes = tb.tb_ternary_linear_workspace("2bit", 2, 20480, 1024)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=DEV)
+    st = tb.tb_ternary_linear_ex(prob.x, tb.TB_BF16, prob.packed, prob.scales, "2bit", 2, 20480,
+                                 1024, prob.signs, torch.empty(2, 20480, device=DEV), tb.TB_FP32,
+                                 ws, ws_bytes, GEMV_TC, check=False)
+    assert st == tb.TB_ERR_SHAPE
+    _check(prob.linear(GEMV), ref, prob.p)
