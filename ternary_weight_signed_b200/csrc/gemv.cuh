@@ -1,331 +1,418 @@
-// Decode GEMV for small M on the 2-bit slot format.
+// Decode GEMV for small M (1 to 4 tokens) on the 2-bit slot format.
 //
 // y[m, n] = sum_g s[n, g] * sum_{k in g} t[n, k] x'[m, k]   (ternary g128;
 // news.ditty.ir second paragraph, ai4coding.ru "What is a ternary model").
 //
-// The ternary multiply is an add/subtract (ai4coding.ru, same section).  Here
-// it is carried out on integers: x' is held per 128-group as 16-bit fixed point
-// q = rint(x' / e_g) split into two int8 planes (hi, lo), and the packed 2-bit
-// word gives the biased codes c = t + 1 directly as bytes, so
-//   sum_k t q = 256 * sum c hi + sum c lo - sum q
-// with four codes per dp4a instruction and exact int32 sums; the group scale
-// s * e_g is applied once per quarter-group in fp32.
+// The ternary multiply is an add/subtract (ai4coding.ru, same section); here
+// it is carried out on integers.  x' is held per 128-group as 16-bit fixed
+// point q = rint(x' / e_g) split into two int8 planes (q = 256 hi + lo), and
+// the packed 2-bit word gives the biased codes c = t + 1 as bytes, so
+//   sum_k t q = 256 * sum c hi + sum c lo - sum q,
+// four codes per dp4a instruction, exact in int32.  The group scale s * e_g
+// is applied in fp32 once per group (per item, see below).
 //
-// Memory side: a persistent grid, one CTA per SM.  CTA c owns a contiguous
-// range of rows, whose packed codes are one contiguous byte range; it streams
-// them as a few large 1-D bulk copies ("segments" of whole rows, up to
-// kSegBytes) into a ring of shared-memory slots, after one copy of all of its
-// scales.  Few, large copies matter: the copy engine's cost is per operation,
-// and small boxes capped the stream far below HBM speed.
+// Two ways to turn a packed word w (16 codes; code 4b + j of the word in bits
+// 8b + 2j of it) into dp4a operands:
+//   shift mode (M >= 2): c_j = (w >> 2j) & 0x03030303, shared by all tokens;
+//   mask mode  (M == 1): w & (0x03030303 << 2j) = 4^j c_j, one instruction;
+//     the four partial sums T_j are 4^j times the true ones, so they are
+//     combined exactly as T_0 + (T_1 >> 2) + (T_2 >> 4) + (T_3 >> 6).
 //
-// Activations: for small M * K the consumer warps compute them in the
-// kernel's prologue (rotation + fixed point, four groups of 128 threads, one
-// 1024-block each at a time) while the first weight segments stream in, so a
-// decode step is one kernel.  Otherwise a prep kernel writes them to the
-// workspace and the consumers load them with plain loads (not through the copy
-// engine, where they would queue behind the weights).
+// Work split.  One CTA of 16 warps per SM; the CTAs own consecutive ranges of
+// R <= 128 weight rows.  K is walked in stages of NB boxes; a box is 128 bytes
+// (512 codes) of each of the CTA's rows, brought by one 2-D TMA copy with the
+// 128-byte swizzle, so a warp whose lanes read the same 16-byte chunk of 32
+// different rows hits every bank group once.  One lane = one weight row, so a
+// row's sum never crosses lanes.  An item is one group (M = 1), half a group
+// (M = 2) or a quarter group (M >= 3) of one stage; a warp takes an item,
+// loads its activation words once into registers (broadcast shared-memory
+// loads: every lane reads the same words) and runs it over all of the CTA's
+// rows, 32 at a time, accumulating each row's fp32 sum in a register.  At the
+// end the warps' per-row partials go through shared memory and are added in a
+// fixed order (bitwise reproducible).
 //
-// Compute side: the work of a segment is split into items of (4 R rows, one
-// 1024-code chunk of K), R = 2 rows per lane for M <= 2 and 1 otherwise.  Items
-// are numbered across segments and consumer warp w takes items w, w + W, ...
-// (W consumer warps), so the split is even for any N and K and every warp
-// starts on the first segment to arrive.  Inside an item lane l owns 128-group
-// l & 7 of the chunk for rows (l >> 3) + 4 i, i < R: the group scale is applied
-// once per 128 codes, the activation words it loads serve R rows, and four
-// independent dp4a chains keep the pipes busy.  The 8 lanes of a row reduce
-// with 3 shuffles and one of them stores the item's sum in a per-(row, chunk)
-// slot in shared memory.  At the end each row's chunk slots are summed in a
-// fixed order, so results are bitwise reproducible.
+// The rotated fixed-point activations are made by prep_gemv_kernel (one
+// 128-thread CTA per token and 1024-block) launched just before.  The decode
+// kernel is launched with programmatic dependent launch: thread 0 issues the
+// weight copies of the first stages (up to the whole ring, which is sized to
+// the SM's shared memory) at once, and only the activation copies wait for the
+// prep kernel.
 #pragma once
 #include "hadamard.cuh"
 #include "tb_device.cuh"
 
 namespace tb {
 
-constexpr int kGemvConsumerWarps = 16;
-constexpr int kGemvThreads = 32 * (kGemvConsumerWarps + 1);
-constexpr int kGemvQuadRows = 4;
 constexpr int kGemvMaxM = 4;
-constexpr int kChunkCodes = 1024;        // K per item
-constexpr int kSegBytes = 32 * 1024;     // target bytes of one weight segment
-constexpr int kGemvMinSlots = 2;
-constexpr int kGemvMaxSlots = 6;
-constexpr int kGemvFwhtBytes = 4 * 1024 * 4;
-constexpr int kGemvFusedMaxBlocks = 16;  // fuse the prologue when M * K/1024 <= this
+constexpr int kGemvWarps = 16;                       // warps per CTA, all consumers
+constexpr int kGemvThreads = 32 * kGemvWarps;
+constexpr int kGemvBoxCodes = 512;                  // K per box: 128 bytes of a row
+constexpr int kGemvMaxNB = 8;                       // boxes per stage at most
+constexpr int kGemvMaxSlots = 12;
+constexpr int kGemvSmemTarget = 227 * 1024;         // one CTA per SM
 
-struct GemvParams {
-  const uint8_t* act;     // prep_gemv output, M rows of gemv_act_row_bytes(K) (when not fused)
-  const void* x;          // [M, K] activations (fused prologue)
-  const int8_t* signs;    // [K] or null (fused prologue)
-  int xt;                 // dtype of x: 0 bf16, 1 fp16, 2 fp32
-  int fused;              // 1: compute the activations in the prologue
-  const uint8_t* packed;  // [N, K/4]
-  const uint16_t* scales; // [N, K/128] fp16 bits
-  void* y;                // [M, N]
-  int N;
-  int K;
-  int seg_rows;           // rows per segment (a multiple of the item height)
-  int nslots;             // ring depth
-  int max_rows;           // largest row range of any CTA (sizes the shared buffers)
-};
+// rows per CTA at most: 32 * kGemvMaxRowTiles(M)
+__host__ __device__ constexpr int gemv_max_row_tiles(int) { return 4; }
+// codes per item
+__host__ __device__ constexpr int gemv_cpi(int M) { return M == 1 ? 128 : (M == 2 ? 64 : 32); }
 
-// Shared-memory layout, in order, each part 128-byte aligned:
-//   act     M * gemv_act_row_bytes(K)
-//   scales  max_rows * K/64 bytes
-//   part    max_rows * (K/1024) * M floats
-//   fwht    4 x 1024 floats (the fused prologue's transforms)
-//   ring    nslots * seg_rows * K/4 bytes
-//   barriers
-__host__ __device__ constexpr int64_t align128(int64_t v) { return (v + 127) & ~int64_t(127); }
-
-__host__ __device__ inline int64_t gemv_smem_bytes(int M, int64_t K, int max_rows, int seg_rows, int nslots) {
-  return 1024 + align128(M * gemv_act_row_bytes(K)) + align128(static_cast<int64_t>(max_rows) * (K / 64)) +
-         align128(static_cast<int64_t>(max_rows) * (K / 1024) * M * 4) + kGemvFwhtBytes +
-         static_cast<int64_t>(nslots) * seg_rows * (K / 4) + 8 * (2 * nslots + 2);
+// Activation block of one stage (what one bulk copy brings):
+//   words[M][4 NB groups][256 B], then info[M][4 NB groups] {float e, int qsum}.
+// Group words: [plane (hi, lo)][i = which 16 codes, 0..7][j = slot, 0..3],
+// 4 bytes each; byte b of word (p, i, j) holds plane p of code 16 i + 4 b + j.
+constexpr int kGemvGroupBytes = 256;
+__host__ __device__ constexpr int64_t gemv_act_stage_bytes(int M, int NB) {
+  return static_cast<int64_t>(M) * NB * 4 * (kGemvGroupBytes + 8);
+}
+__host__ __device__ constexpr int64_t gemv_nstage(int64_t K, int NB) {
+  return (K / kGemvBoxCodes + NB - 1) / NB;
+}
+// Workspace bound valid for every NB <= kGemvMaxNB.
+__host__ __device__ constexpr int64_t gemv_ws_bytes(int64_t M, int64_t K) {
+  return (K / kGemvBoxCodes + kGemvMaxNB) * M * 4 * (kGemvGroupBytes + 8);
 }
 
+struct GemvParams {
+  const uint8_t* act;      // prep_gemv_kernel output, stage blocks
+  const uint16_t* scales;  // [N, K/128] fp16 bits
+  void* y;                 // [M, N]
+  int N, K;
+  int R;                   // rows per CTA (box height)
+  int RT;                  // row tiles of 32 covering R
+  int NB;                  // boxes per stage
+  int nstage;
+  int nslots;
+  int box_stride;          // bytes between the boxes of a slot (1 KB multiple)
+  int slot_bytes;          // boxes + activation block
+  int sc_bytes;            // shared-memory bytes for the CTA's scales
+};
+
+__host__ __device__ constexpr int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ constexpr int64_t align128(int64_t v) { return align_up(v, 128); }
+
+// Shared memory: [1 KB alignment slack] scales | ring of slots | barriers and
+// per-slot counters.
+__host__ __device__ inline int64_t gemv_smem_bytes(int64_t sc_bytes, int64_t slot_bytes, int nslots) {
+  return 1024 + sc_bytes + slot_bytes * nslots + 8 * (kGemvMaxSlots + 1) + 4 * kGemvMaxSlots;
+}
+
+// Activation prep: grid (K/1024, M), 128 threads per (1024-block, token);
+// thread t holds elements 8t .. 8t+7 of the block (the 128-thread block
+// transform of hadamard.cuh), so a 128-group is 16 threads and thread pair
+// (2i, 2i+1) of a group holds its 16-code word i.  Launched with programmatic
+// dependent launch: it waits for the previous kernel on the stream (which may
+// have produced x, or may still be reading this workspace) before touching
+// either.
+template <typename TIn>
+__global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restrict__ x,
+                                                              const int8_t* __restrict__ signs,
+                                                              uint8_t* __restrict__ ws, int K, int NB) {
+  __shared__ float sm[kHB];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int blk = blockIdx.x, m = blockIdx.y, M = gridDim.y, t = threadIdx.x;
+  float v[8];
+  load_rotated8<TIn>(x, signs, m, blk, K, v, sm);
+  float mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float e = mx / kQMax;
+  const float inv = mx > 0.f ? kQMax / mx : 0.f;
+  int hi[8], lo[8];
+  int qs = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int q = max(-32512, min(32512, __float2int_rn(v[i] * inv)));
+    qs += q;
+    hi[i] = (q + 128) >> 8;
+    lo[i] = q - (hi[i] << 8);
+  }
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+  // Byte b of word (plane, i, j) is code 16 i + 4 b + j: the even thread of the
+  // pair supplies bytes 0, 1 (its elements j and 4 + j), the odd one bytes 2, 3.
+  // The even thread writes the hi plane's four words, the odd one the lo plane's.
+  const int u = t & 15, h = u & 1, wi = u >> 1;
+  uint32_t word[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t hh = (static_cast<uint32_t>(hi[j]) & 0xFFu) | ((static_cast<uint32_t>(hi[4 + j]) & 0xFFu) << 8);
+    const uint32_t hl = (static_cast<uint32_t>(lo[j]) & 0xFFu) | ((static_cast<uint32_t>(lo[4 + j]) & 0xFFu) << 8);
+    const uint32_t recv = __shfl_xor_sync(0xffffffffu, h ? hh : hl, 1);
+    word[j] = h ? (recv | (hl << 16)) : (hh | (recv << 16));
+  }
+  const int g = blk * 8 + (t >> 4);  // global group index
+  const int s = g / (4 * NB), gs = g % (4 * NB);
+  uint8_t* blkbase = ws + static_cast<int64_t>(s) * gemv_act_stage_bytes(M, NB);
+  uint8_t* gw = blkbase + (static_cast<int64_t>(m) * 4 * NB + gs) * kGemvGroupBytes;
+  *reinterpret_cast<uint4*>(gw + h * 128 + wi * 16) = make_uint4(word[0], word[1], word[2], word[3]);
+  if (u == 0) {
+    int2 inf;
+    inf.x = __float_as_int(e);
+    inf.y = qs;
+    reinterpret_cast<int2*>(blkbase + static_cast<int64_t>(M) * 4 * NB * kGemvGroupBytes)[m * 4 * NB + gs] = inf;
+  }
+}
+
+// Integer group sum  sum_k c_k q_k  of one item for one token, mask mode (a
+// whole group: 8 packed words, 64 activation words A[p][i][j] at 32 p + 4 i + j).
+__device__ __forceinline__ int gemv_item_mask(const uint32_t (&w)[8], const uint32_t (&A)[64]) {
+  int th[4] = {0, 0, 0, 0}, tl[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t c = w[i] & (0x03030303u << (2 * j));
+      th[j] = dp4a_us(c, A[4 * i + j], th[j]);
+      tl[j] = dp4a_us(c, A[32 + 4 * i + j], tl[j]);
+    }
+  }
+  int t[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) t[j] = th[j] * 256 + tl[j];
+  return t[0] + (t[1] >> 2) + (t[2] >> 4) + (t[3] >> 6);
+}
+
+// Copies stage s into slot slot_i (= s % nslots): the NB weight boxes and the activation
+// block, all completing on the slot's full barrier.  With act == false the
+// activation copy is left for later (it waits for the prep kernel).
+__device__ __forceinline__ void gemv_issue_stage(const CUtensorMap* tm, const GemvParams& p, uint8_t* ring,
+                                                 uint64_t* full, int s, int slot_i, int r0, uint32_t wbytes,
+                                                 uint32_t abytes, bool weights, bool act) {
+  uint8_t* slot = ring + static_cast<int64_t>(slot_i) * p.slot_bytes;
+  if (weights) {
+    mbar_arrive_expect_tx(&full[slot_i], wbytes + abytes);
+    for (int b = 0; b < p.NB; ++b) tma_load_2d(slot + b * p.box_stride, tm, (s * p.NB + b) * 128, r0, &full[slot_i]);
+  }
+  if (act)
+    bulk_load(slot + p.NB * p.box_stride, p.act + static_cast<int64_t>(s) * abytes, abytes, &full[slot_i]);
+}
+
+// One CTA: rows [blockIdx.x * R, +R), all of K.  Sixteen warps, no dedicated
+// producer: thread 0 issues the first nslots stages, and afterwards the last
+// warp to finish with a stage refills its slot with the stage nslots later.
 template <int M, typename TOut>
-__global__ void __launch_bounds__(kGemvThreads, 1) gemv_2bit_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    gemv_2bit_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
+  constexpr int CPI = gemv_cpi(M);  // codes per item
+  constexpr int PPG = 128 / CPI;    // items per group
+  constexpr int WPI = CPI / 16;     // packed 32-bit words per row and item
+  constexpr int AW = 2 * WPI * 4;   // activation words per token and item
+  constexpr int RTM = gemv_max_row_tiles(M);
+  constexpr int NW = kGemvWarps;
+
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
-  const int K = p.K;
-  const int C = K / kChunkCodes;     // chunks per row
-  const int64_t RB = K / 4;          // packed bytes per row
-  const int G = K / 128;
-  const int64_t act_bytes = static_cast<int64_t>(M) * gemv_act_row_bytes(K);
-
-  // this CTA's rows
-  const int r0 = static_cast<int>((static_cast<int64_t>(p.N) * blockIdx.x) / gridDim.x);
-  const int r1 = static_cast<int>((static_cast<int64_t>(p.N) * (blockIdx.x + 1)) / gridDim.x);
-  const int nrows = r1 - r0;
-  const int nseg = (nrows + p.seg_rows - 1) / p.seg_rows;
-
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* act = base;
-  __half* sc = reinterpret_cast<__half*>(act + align128(act_bytes));
-  float* acc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sc) +
-                                        align128(static_cast<int64_t>(p.max_rows) * (K / 64)));
-  float* fsm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(acc) +
-                                        align128(static_cast<int64_t>(p.max_rows) * C * M * 4));
-  uint8_t* ring = reinterpret_cast<uint8_t*>(fsm) + kGemvFwhtBytes;
-  const int64_t slot_bytes = static_cast<int64_t>(p.seg_rows) * RB;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + p.nslots * slot_bytes);
-  uint64_t* empty = full + p.nslots;
-  uint64_t* sc_bar = empty + p.nslots;  // this CTA's scales
+  const __half* sc = reinterpret_cast<const __half*>(base);
+  uint8_t* ring = base + p.sc_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + static_cast<int64_t>(p.nslots) * p.slot_bytes);
+  uint64_t* sc_bar = full + kGemvMaxSlots;
+  uint32_t* done = reinterpret_cast<uint32_t*>(sc_bar + 1);  // warps finished per slot
 
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  const int G = p.K / 128;
+  const int r0 = blockIdx.x * p.R;
+  const int nrows = min(p.R, p.N - r0);
+  const int IPS = p.NB * 4 * PPG;          // items per stage
+  const int Q = IPS >= NW ? 1 : NW / IPS;  // stages worked on at once
+  const int WPS = IPS >= NW ? NW : IPS;    // warps per stage
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t wbytes = static_cast<uint32_t>(p.NB) * static_cast<uint32_t>(p.R) * 128u;
+  const uint32_t abytes = static_cast<uint32_t>(gemv_act_stage_bytes(M, p.NB));
+  const int act_off = p.NB * p.box_stride;  // activation block inside a slot
+  const int pre = min(p.nslots, p.nstage);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.nslots; ++s) {
+    for (int s = 0; s < kGemvMaxSlots; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGemvConsumerWarps);
+      done[s] = 0;
     }
     mbar_init(sc_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
-
-  if (warp == kGemvConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint8_t* src = p.packed + static_cast<int64_t>(r0) * RB;
-      const uint32_t sbytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(K / 64);
-      mbar_arrive_expect_tx(sc_bar, sbytes);
-      bulk_load(sc, p.scales + static_cast<int64_t>(r0) * G, sbytes, sc_bar);
-      for (int s = 0; s < nseg; ++s) {
-        const int slot = s % p.nslots;
-        if (s >= p.nslots && !mbar_wait(&empty[slot], ((s / p.nslots) & 1) ^ 1, FAULT_WAIT_EMPTY)) break;
-        const int rows = min(p.seg_rows, nrows - s * p.seg_rows);
-        const uint32_t bytes = static_cast<uint32_t>(rows * RB);
-        mbar_arrive_expect_tx(&full[slot], bytes);
-        bulk_load(ring + slot * slot_bytes, src + static_cast<int64_t>(s) * p.seg_rows * RB, bytes, &full[slot]);
-      }
-    }
-    return;
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tm_w);
+    const uint32_t sbytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(G * 2);
+    mbar_arrive_expect_tx(sc_bar, sbytes);
+    bulk_load(base, p.scales + static_cast<int64_t>(r0) * G, sbytes, sc_bar);
+    // weights do not depend on the prep kernel; its activation blocks do
+    for (int s = 0; s < pre; ++s) gemv_issue_stage(&tm_w, p, ring, full, s, s, r0, wbytes, abytes, true, false);
+    pdl_wait();
+    for (int s = 0; s < pre; ++s) gemv_issue_stage(&tm_w, p, ring, full, s, s, r0, wbytes, abytes, false, true);
   }
+  // The other threads wait here (a hardware barrier, no issue slots taken)
+  // while thread 0 waits for the prep kernel: a CTA that starts early, next to
+  // one of the previous call still computing on the same SM, stays idle.
+  __syncthreads();
 
-  // -------------------------------------------------------------- consumers
-  constexpr int R = M <= 2 ? 2 : 1;           // rows per lane
-  constexpr int IR = 4 * R;                   // rows per item
-  const int g = lane & 7;                     // 128-group of the chunk this lane owns
-  const int rl = lane >> 3;                   // row within each 4-row slice
-  pdl_wait();  // x (fused) or the prep kernel's output must be complete
-  if (p.fused) {
-    // activations of all M tokens: rotation, 16-bit fixed point per 128-group,
-    // planes laid out exactly as prep_gemv_kernel writes them
-    const int cg = warp >> 2, t = threadIdx.x & 127;
-    float* gsm = fsm + cg * 1024;
-    const int nblk = K / kHB;
-    for (int pi = cg; pi < M * nblk; pi += 4) {
-      const int m = pi / nblk, blk = pi - m * nblk;
-      const int64_t k0 = static_cast<int64_t>(blk) * kHB + 8 * t;
-      float v[8];
-      if (p.xt == 0)
-        load8<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(p.x) + static_cast<int64_t>(m) * K + k0, v);
-      else if (p.xt == 1)
-        load8<__half>(static_cast<const __half*>(p.x) + static_cast<int64_t>(m) * K + k0, v);
-      else
-        load8<float>(static_cast<const float*>(p.x) + static_cast<int64_t>(m) * K + k0, v);
-      if (p.signs != nullptr) {
-        float dsg[8];
-        load_signs8(p.signs + k0, dsg);
+  float acc[M][RTM];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] *= dsg[i];
-        fwht1024_group(v, gsm, t, 2 + cg);
+  for (int m = 0; m < M; ++m)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] *= kHNorm;
-      }
-      float mx = 0.f;
+    for (int t = 0; t < RTM; ++t) acc[m][t] = 0.f;
+  // This lane's rows are 32 t + lane (rows past R repeat row R - 1; their sums
+  // are discarded): byte offsets of the rows in a box and of their scales.  The
+  // 128-byte swizzle XORs the 16-byte chunk index with the row index mod 8,
+  // which is lane & 7 for every tile.
+  int roff[RTM], soff[RTM];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float e = mx / kQMax;
-      const float inv = mx > 0.f ? kQMax / mx : 0.f;
-      int qs = 0;
-      uint8_t* hrow = act + static_cast<int64_t>(m) * gemv_act_row_bytes(K) + static_cast<int64_t>(blk) * kHB;
-      const int c = t >> 1, h = t & 1;
-      const int wbase = 128 * (c & 7) + 16 * (c >> 3);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int qi = max(-32512, min(32512, __float2int_rn(v[i] * inv)));
-        qs += qi;
-        const int hi = (qi + 128) >> 8;
-        const int lo = qi - (hi << 8);
-        const int b = 2 * h + (i >> 2), j = i & 3;
-        hrow[wbase + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(hi));
-        hrow[K + wbase + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(lo));
-      }
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
-      if ((t & 15) == 0) {
-        int2 inf;
-        inf.x = __float_as_int(e);
-        inf.y = qs;
-        reinterpret_cast<int2*>(act + static_cast<int64_t>(m) * gemv_act_row_bytes(K) + 2 * K)[blk * 8 + (t >> 4)] = inf;
-      }
-    }
-  } else {
-    const int64_t n16 = act_bytes / 16;
-    for (int64_t i = threadIdx.x; i < n16; i += 32 * kGemvConsumerWarps)
-      reinterpret_cast<uint4*>(act)[i] = reinterpret_cast<const uint4*>(p.act)[i];
+  for (int t = 0; t < RTM; ++t) {
+    roff[t] = min(32 * t + lane, p.R - 1) * 128;
+    soff[t] = min(32 * t + lane, nrows - 1) * G;
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(32 * kGemvConsumerWarps) : "memory");
-  bool ok = mbar_wait(sc_bar, 0, FAULT_WAIT_ACT);
-  int item_base = 0;  // number of the first item of the current segment
-  for (int s = 0; s < nseg && ok; ++s) {
-    const int slot = s % p.nslots;
-    const int srow0 = s * p.seg_rows;  // first row of the segment, relative to r0
-    const int rows = min(p.seg_rows, nrows - srow0);
-    const int nsl = (rows + IR - 1) / IR;  // row slices of IR rows
-    const int nitems = nsl * C;
-    int first = (warp - item_base) % kGemvConsumerWarps;
-    if (first < 0) first += kGemvConsumerWarps;
-    // Every warp waits for every segment, even one with no items in it: its
-    // release of the slot must count toward this fill of the slot, not a later one.
-    if (!mbar_wait(&full[slot], (s / p.nslots) & 1, FAULT_WAIT_FULL)) {
+  const int sw = lane & 7;
+
+  const int it0 = IPS >= NW ? warp : warp % IPS;
+  const int q = IPS >= NW ? 0 : warp / IPS;
+  bool ok = mbar_wait_backoff(sc_bar, 0, FAULT_WAIT_ACT);
+  // stage s lives in slot s % nslots with barrier phase (s / nslots) & 1;
+  // nslots is a multiple of Q, so stepping s by Q wraps the slot exactly
+  int slot_i = q;
+  uint32_t phase = 0;
+  for (int s = q; s < p.nstage && ok; s += Q) {
+    if (!mbar_wait_backoff(&full[slot_i], phase, FAULT_WAIT_FULL)) {
       ok = false;
       break;
     }
-    const uint8_t* seg = ring + slot * slot_bytes;
-    int sl = first / C;
-    int kc = first - sl * C;
-    for (int it = first; it < nitems; it += kGemvConsumerWarps) {
-      const int grp = kc * 8 + g;  // group index within the row
-      const uint8_t* ga = act + kc * kChunkCodes + g * 16;  // word 0 of this group, hi plane, token 0
-      int qsum[M];
+    const uint8_t* slot = ring + slot_i * p.slot_bytes;
+    const uint8_t* act = slot + act_off;
+    for (int it = it0; it < IPS; it += NW) {
+      const int gs = it / PPG, pt = it % PPG;  // group within the stage, part of the group
+      const int g = s * 4 * p.NB + gs;          // global group
+      if (g >= G) continue;                     // past K in the last stage
+      const int b = gs >> 2, gl = gs & 3;       // box, group within the box
+      // activation words and {e, qsum} of this item for every token (broadcast loads)
+      uint32_t A[M][AW];
       float e[M];
+      int qs[M];
 #pragma unroll
       for (int m = 0; m < M; ++m) {
-        const int2 inf = *reinterpret_cast<const int2*>(act + static_cast<int64_t>(m) * gemv_act_row_bytes(K) +
-                                                        2 * K + 8 * grp);
-        e[m] = __int_as_float(inf.x);
-        qsum[m] = inf.y;
-      }
-      // rows of this lane (relative to the segment) and their packed words
-      int srow[R];
-      bool live[R];
-      uint4 wv[R][2];
+        const uint8_t* gw = act + (m * 4 * p.NB + gs) * kGemvGroupBytes;
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
-        srow[i] = sl * IR + 4 * i + rl;
-        live[i] = srow[i] < rows;
-        const uint8_t* wp = seg + static_cast<int64_t>(live[i] ? srow[i] : 0) * RB + kc * 256 + g * 32;
-        wv[i][0] = *reinterpret_cast<const uint4*>(wp);
-        wv[i][1] = *reinterpret_cast<const uint4*>(wp + 16);
-      }
-      int dh[R][M][4], dl[R][M][4];
+        for (int pl = 0; pl < 2; ++pl) {
+          const uint4* src = reinterpret_cast<const uint4*>(gw + pl * 128 + pt * CPI);
 #pragma unroll
-      for (int i = 0; i < R; ++i)
-#pragma unroll
-        for (int m = 0; m < M; ++m)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            dh[i][m][j] = 0;
-            dl[i][m][j] = 0;
+          for (int v = 0; v < AW / 8; ++v) {
+            const uint4 u4 = src[v];
+            A[m][pl * (AW / 2) + 4 * v] = u4.x;
+            A[m][pl * (AW / 2) + 4 * v + 1] = u4.y;
+            A[m][pl * (AW / 2) + 4 * v + 2] = u4.z;
+            A[m][pl * (AW / 2) + 4 * v + 3] = u4.w;
           }
-#pragma unroll
-      for (int wd = 0; wd < 8; ++wd) {  // 16-code word of the group
-        uint4 ahi[M], alo[M];
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const uint8_t* am = ga + static_cast<int64_t>(m) * gemv_act_row_bytes(K);
-          ahi[m] = *reinterpret_cast<const uint4*>(am + 128 * wd);
-          alo[m] = *reinterpret_cast<const uint4*>(am + K + 128 * wd);
         }
+        const int2 inf = reinterpret_cast<const int2*>(act + M * 4 * p.NB * kGemvGroupBytes)[m * 4 * p.NB + gs];
+        e[m] = __int_as_float(inf.x);
+        qs[m] = pt == 0 ? inf.y : 0;
+      }
+      const uint8_t* box = slot + b * p.box_stride;
+      // the item's packed words of one row: chunk(s) of the row's 128 bytes
+      int c0, c1 = 0, h8 = 0;
+      if constexpr (WPI == 8) {
+        c0 = ((2 * gl) ^ sw) << 4;
+        c1 = ((2 * gl + 1) ^ sw) << 4;
+      } else if constexpr (WPI == 4) {
+        c0 = ((2 * gl + pt) ^ sw) << 4;
+      } else {
+        c0 = ((2 * gl + (pt >> 1)) ^ sw) << 4;
+        h8 = 8 * (pt & 1);
+      }
+      uint32_t nx[WPI];  // next tile's words, loaded one tile ahead
+      auto load_words = [&](int t, uint32_t (&w)[WPI]) {
+        const uint8_t* rp = box + roff[t];
+        if constexpr (WPI == 8) {
+          const uint4 u0 = *reinterpret_cast<const uint4*>(rp + c0);
+          const uint4 u1 = *reinterpret_cast<const uint4*>(rp + c1);
+          w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+          w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
+        } else if constexpr (WPI == 4) {
+          const uint4 u0 = *reinterpret_cast<const uint4*>(rp + c0);
+          w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+        } else {
+          const uint2 u0 = *reinterpret_cast<const uint2*>(rp + c0 + h8);
+          w[0] = u0.x; w[1] = u0.y;
+        }
+      };
+      load_words(0, nx);
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
-          const uint32_t w = (&wv[i][wd >> 2].x)[wd & 3];
+      for (int t = 0; t < RTM; ++t) {
+        if (t < p.RT) {
+          uint32_t w[WPI];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t c = (w >> (2 * j)) & 0x03030303u;
+          for (int i = 0; i < WPI; ++i) w[i] = nx[i];
+          if (t + 1 < RTM && t + 1 < p.RT) load_words(t + 1, nx);
+          const float s_rg = __half2float(sc[soff[t] + g]);
+          if constexpr (M == 1) {
+            const int tot = gemv_item_mask(w, A[0]) - qs[0];
+            acc[0][t] = fmaf(__int2float_rn(tot), s_rg * e[0], acc[0][t]);
+          } else {
+            int h[M], l[M];
 #pragma unroll
             for (int m = 0; m < M; ++m) {
-              dh[i][m][j] = dp4a_us(c, (&ahi[m].x)[j], dh[i][m][j]);
-              dl[i][m][j] = dp4a_us(c, (&alo[m].x)[j], dl[i][m][j]);
+              h[m] = 0;
+              l[m] = 0;
             }
+#pragma unroll
+            for (int i = 0; i < WPI; ++i) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t c = (w[i] >> (2 * j)) & 0x03030303u;
+#pragma unroll
+                for (int m = 0; m < M; ++m) {
+                  h[m] = dp4a_us(c, A[m][4 * i + j], h[m]);
+                  l[m] = dp4a_us(c, A[m][AW / 2 + 4 * i + j], l[m]);
+                }
+              }
+            }
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+              acc[m][t] = fmaf(__int2float_rn(h[m] * 256 + l[m] - qs[m]), s_rg * e[m], acc[m][t]);
           }
         }
       }
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const float s_rg = live[i] ? __half2float(sc[static_cast<int64_t>(srow0 + srow[i]) * G + grp]) : 0.f;
-        float v[M];
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const int hi = (dh[i][m][0] + dh[i][m][1]) + (dh[i][m][2] + dh[i][m][3]);
-          const int lo = (dl[i][m][0] + dl[i][m][1]) + (dl[i][m][2] + dl[i][m][3]);
-          v[m] = __int2float_rn(hi * 256 + lo - qsum[m]) * (s_rg * e[m]);
-          v[m] += __shfl_xor_sync(0xffffffffu, v[m], 1);
-          v[m] += __shfl_xor_sync(0xffffffffu, v[m], 2);
-          v[m] += __shfl_xor_sync(0xffffffffu, v[m], 4);
-        }
-        if (live[i] && g < M) {
-          float o = v[0];
-#pragma unroll
-          for (int m = 1; m < M; ++m)
-            if (g == m) o = v[m];
-          acc[((srow0 + srow[i]) * C + kc) * M + g] = o;
-        }
-      }
-      kc += kGemvConsumerWarps;
-      while (kc >= C) {
-        kc -= C;
-        ++sl;
+    }
+    // the last warp out of this stage refills the slot
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&done[slot_i], 1u) == static_cast<uint32_t>(WPS - 1)) {
+        __threadfence_block();
+        done[slot_i] = 0;
+        if (s + p.nslots < p.nstage)
+          gemv_issue_stage(&tm_w, p, ring, full, s + p.nslots, slot_i, r0, wbytes, abytes, true, true);
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
-    item_base += nitems;
+    slot_i += Q;
+    if (slot_i >= p.nslots) {
+      slot_i -= p.nslots;
+      phase ^= 1u;
+    }
   }
-  // all consumer warps done: write this CTA's rows
-  asm volatile("bar.sync 1, %0;" ::"n"(32 * kGemvConsumerWarps) : "memory");
+  // every copy must have landed before the ring is reused: wait for the last
+  // stage of every slot (already complete unless a wait above gave up)
+  if (threadIdx.x == 0) {
+    for (int s = max(0, p.nstage - p.nslots); s < p.nstage; ++s)
+      if (!mbar_wait(&full[s % p.nslots], (s / p.nslots) & 1, FAULT_WAIT_FULL)) break;
+  }
+  // park the per-warp row partials in the ring and add them in a fixed order
+  __syncthreads();
+  float* part = reinterpret_cast<float*>(ring);
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int t = 0; t < RTM; ++t)
+      if (t < p.RT) part[((m * p.RT + t) * 32 + lane) * NW + warp] = acc[m][t];
+  __syncthreads();
   TOut* y = reinterpret_cast<TOut*>(p.y);
-  for (int i = threadIdx.x; i < nrows * M; i += 32 * kGemvConsumerWarps) {
-    const int lr = i / M, m = i - lr * M;
-    float v = 0.f;
-    for (int kc = 0; kc < C; ++kc) v += acc[(lr * C + kc) * M + m];
-    y[static_cast<int64_t>(m) * p.N + r0 + lr] = from_f32<TOut>(v);
+  for (int idx = threadIdx.x; idx < M * nrows; idx += kGemvThreads) {
+    const int m = idx / nrows, r = idx - m * nrows;
+    const float* src = part + (m * p.RT * 32 + r) * NW;
+    float sum = 0.f;
+    for (int i = 0; i < NW; ++i) sum += src[i];
+    y[static_cast<int64_t>(m) * p.N + r0 + r] = from_f32<TOut>(sum);
   }
 }
 

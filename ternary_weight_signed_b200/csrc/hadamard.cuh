@@ -198,82 +198,10 @@ __global__ void __launch_bounds__(kHThreads) rotate_kernel(const TIn* x, TOut* y
 }
 
 // ---------------------------------------------------------------------------
-// GEMV activation prep.  Per token row, the workspace holds
-//   hi[K] int8 | lo[K] int8 | info[K/128] {float e, int qsum}
-// (2 K + K/16 bytes).  For each 128-group g: e_g = max|x'_g| / 32512,
-// q = rint(x' / e_g) in [-32512, 32512], q = 256 hi + lo with hi in
-// [-127, 127], lo in [-128, 127]; info holds e_g and the sum of q over the group.
-// Within each 16-code word the planes are permuted so that byte 4j + b holds
-// code k = 4b + j: then ((w >> 2j) & 0x03030303) of a packed 2-bit word and
-// activation word j line up byte for byte in dp4a.  Within each 1024-code
-// block the 16-byte words are stored word-major ([word wd][group g]): word wd
-// of group g sits at 128 wd + 16 g, so the 8 lanes that read word wd of the 8
-// groups of a block touch 128 contiguous bytes (no shared-memory bank conflict).
+// 16-bit fixed point of the rotated activations used by the decode kernels:
+// per 128-group e_g = max|x'_g| / kQMax, q = rint(x' / e_g) in [-32512, 32512],
+// q = 256 hi + lo with hi = (q + 128) >> 8 in [-127, 127], lo in [-128, 127].
 constexpr float kQMax = 32512.0f;
-
-__host__ __device__ constexpr int64_t gemv_act_row_bytes(int64_t K) { return 2 * K + K / 16; }
-
-template <typename TIn>
-__global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restrict__ x,
-                                                              const int8_t* __restrict__ signs,
-                                                              uint8_t* __restrict__ ws, int64_t K) {
-  __shared__ float sm[kHB];
-  __shared__ uint2 hi_s[128];
-  __shared__ uint2 lo_s[128];
-  pdl_launch_dependents();
-  const int64_t row = blockIdx.x;
-  const int blk = blockIdx.y;
-  const int t = threadIdx.x;
-  float v[8];
-  load_rotated8<TIn>(x, signs, row, blk, K, v, sm);
-  // group max over 16 threads (128 elements)
-  float mx = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
-#pragma unroll
-  for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const float e = mx / kQMax;
-  const float inv = mx > 0.f ? kQMax / mx : 0.f;
-  int q[8];
-  int qs = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int qi = __float2int_rn(v[i] * inv);
-    qi = max(-32512, min(32512, qi));
-    q[i] = qi;
-    qs += qi;
-  }
-  qs += __shfl_xor_sync(0xffffffffu, qs, 1);  // over the group's 16 threads
-  qs += __shfl_xor_sync(0xffffffffu, qs, 2);
-  qs += __shfl_xor_sync(0xffffffffu, qs, 4);
-  qs += __shfl_xor_sync(0xffffffffu, qs, 8);
-  // Thread pair (2c, 2c+1) holds chunk c; element i of thread half h is code
-  // k = 8h + i = 4b + j with b = 2h + i/4, j = i%4 -> permuted byte 4j + b.
-  __syncthreads();  // sm reuse guard not needed for hi_s/lo_s, keep ordering simple
-  uint8_t* hb = reinterpret_cast<uint8_t*>(hi_s);
-  uint8_t* lb = reinterpret_cast<uint8_t*>(lo_s);
-  const int c = t >> 1, h = t & 1;           // 16-code word c of the block
-  const int wbase = 128 * (c & 7) + 16 * (c >> 3);  // word (c & 7) of group (c >> 3)
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int hi = (q[i] + 128) >> 8;
-    const int lo = q[i] - (hi << 8);
-    const int b = 2 * h + (i >> 2), j = i & 3;
-    hb[wbase + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(hi));
-    lb[wbase + 4 * j + b] = static_cast<uint8_t>(static_cast<int8_t>(lo));
-  }
-  __syncthreads();
-  uint8_t* base = ws + row * gemv_act_row_bytes(K);
-  const int64_t k0 = static_cast<int64_t>(blk) * kHB;
-  reinterpret_cast<uint2*>(base + k0)[t] = hi_s[t];
-  reinterpret_cast<uint2*>(base + K + k0)[t] = lo_s[t];
-  if ((t & 15) == 0) {
-    int2 inf;
-    inf.x = __float_as_int(e);
-    inf.y = qs;
-    reinterpret_cast<int2*>(base + 2 * K)[(k0 >> 7) + (t >> 4)] = inf;
-  }
-}
 
 // Rotated (or converted) activations in fp32 / fp16 for the plain and the
 // tensor-core kernels: grid (M, K/1024).

@@ -94,6 +94,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
+// The same, for waiters that are not on the critical path of a copy: after a
+// failed poll the thread sleeps briefly, so that warps waiting for data leave
+// the issue slots to warps that compute.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, uint32_t fault) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    __nanosleep(100);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      record_fault(fault);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 // 2-D tiled load of one box into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,

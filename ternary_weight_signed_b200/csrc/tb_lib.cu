@@ -72,8 +72,15 @@ tb_status allow_smem(F* fn, const DevInfo* d) {
                        (static_cast<uint64_t>(dev) << 56);
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_smem_set.count(key)) return TB_OK;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, d->max_smem_optin) !=
-      cudaSuccess) {
+  // all of these kernels stage through shared memory: ask for the largest carveout
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  const int dyn_max = d->max_smem_optin - static_cast<int>(fa.sharedSizeBytes);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) != cudaSuccess ||
+      cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) {
     cudaGetLastError();
     return TB_ERR_CUDA;
   }
@@ -194,6 +201,8 @@ size_t workspace_bytes(int64_t M, int64_t K) {
   size_t b = static_cast<size_t>(4) * static_cast<size_t>(M) * static_cast<size_t>(K);
   const size_t g = static_cast<size_t>(gtc_ws_bytes(M, K));  // tensor-core decode activations
   if (g > b) b = g;
+  const size_t v = static_cast<size_t>(gemv_ws_bytes(M, K));  // decode activation words
+  if (v > b) b = v;
   return (b + 255) & ~static_cast<size_t>(255);
 }
 
@@ -203,30 +212,56 @@ bool fast_aligned(const LinearArgs& a) {
 }
 
 struct GemvPlan {
-  int grid, max_rows, seg_rows, nslots;
+  int grid, R, RT, NB, nstage, nslots, box_stride, slot_bytes, sc_bytes;
   size_t smem;
 };
 
 // Geometry of the decode kernel for these sizes on a device with `sm_count`
 // SMs and `max_smem` bytes of shared memory per block; false if it does not fit.
 bool gemv_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, GemvPlan* out) {
-  if (M < 1 || M > kGemvMaxM || K % 1024 != 0 || N < 1) return false;
+  if (M < 1 || M > kGemvMaxM || K % 1024 != 0 || K < 1024 || N < 1 || sm_count < 1) return false;
   GemvPlan pl;
-  pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
-  pl.max_rows = static_cast<int>((N + pl.grid - 1) / pl.grid);
-  const int64_t rb = K / 4;
-  const int64_t ir = M <= 2 ? 8 : 4;  // rows per work item (see gemv_2bit_kernel)
-  int64_t sr = ir * (kSegBytes / (ir * rb));
-  if (sr < ir) sr = ir;
-  pl.seg_rows = static_cast<int>(sr);
-  const int64_t fixed = gemv_smem_bytes(static_cast<int>(M), K, pl.max_rows, pl.seg_rows, 0) + 8 * 2 * kGemvMaxSlots;
-  int64_t ns = (static_cast<int64_t>(max_smem) - fixed) / (sr * rb);
+  const int64_t rmax = 32 * gemv_max_row_tiles(static_cast<int>(M));
+  int64_t R = (N + sm_count - 1) / sm_count;
+  if (R > rmax) R = rmax;
+  pl.R = static_cast<int>(R);
+  pl.RT = static_cast<int>((R + 31) / 32);
+  pl.grid = static_cast<int>((N + R - 1) / R);
+  const int64_t G = K / 128;
+  // boxes per stage: enough that one stage moves >= 12 KB of weights
+  const int64_t boxes = K / kGemvBoxCodes;
+  int NB = 1;
+  while (NB < kGemvMaxNB && NB < boxes && static_cast<int64_t>(NB) * R * 128 < 12 * 1024) NB *= 2;
+  pl.NB = NB;
+  pl.nstage = static_cast<int>(gemv_nstage(K, NB));
+  pl.box_stride = static_cast<int>(align_up(R * 128, 1024));
+  pl.slot_bytes = static_cast<int>(align_up(static_cast<int64_t>(NB) * pl.box_stride +
+                                                gemv_act_stage_bytes(static_cast<int>(M), NB), 1024));
+  pl.sc_bytes = static_cast<int>(align_up(R * G * 2, 1024));
+  // the scales of the CTA arrive on one barrier: < 2^20 bytes
+  if (R * G * 2 >= (int64_t(1) << 20)) return false;
+  const int64_t part = M * pl.RT * 32 * kGemvWarps * 4;  // row partials, parked in the ring at the end
+  const int64_t budget = std::min<int64_t>(max_smem, kGemvSmemTarget);
+  int64_t ns = (budget - gemv_smem_bytes(pl.sc_bytes, 0, 0)) / pl.slot_bytes;
   if (ns > kGemvMaxSlots) ns = kGemvMaxSlots;
-  if (ns < kGemvMinSlots) return false;
-  // the activations + scales arrive on one barrier whose byte count is < 2^20
-  if (M * gemv_act_row_bytes(K) + static_cast<int64_t>(pl.max_rows) * (K / 64) >= (int64_t(1) << 20)) return false;
+  if (ns >= pl.nstage) {
+    ns = pl.nstage;  // every stage has a slot of its own: no slot is reused
+  } else {
+    // When the warps split into Q groups that take alternate stages, each slot
+    // must belong to one group (nslots a multiple of Q): a warp may then wait
+    // on a slot's barrier at most one phase ahead of it.
+    const int ips = NB * 4 * (128 / gemv_cpi(static_cast<int>(M)));
+    const int qg = ips >= kGemvWarps ? 1 : kGemvWarps / ips;
+    ns -= ns % qg;
+    if (ns < qg || ns < 2) return false;
+  }
+  // the row partials are parked in the ring at the end
+  while (ns * pl.slot_bytes < part && ns < kGemvMaxSlots) ++ns;
+  if (ns * pl.slot_bytes < part) return false;
   pl.nslots = static_cast<int>(ns);
-  pl.smem = static_cast<size_t>(gemv_smem_bytes(static_cast<int>(M), K, pl.max_rows, pl.seg_rows, pl.nslots));
+  const int64_t smem = gemv_smem_bytes(pl.sc_bytes, pl.slot_bytes, pl.nslots);
+  if (smem > max_smem) return false;
+  pl.smem = static_cast<size_t>(smem);
   *out = pl;
   return true;
 }
@@ -307,18 +342,15 @@ int auto_path(const LinearArgs& a) {
 }
 
 // ------------------------------------------------------------------ linear: GEMV
-// The fused kernel has no prep kernel before it to overlap with; launching it
-// without programmatic serialization keeps it ordered after all prior work.
+// Both kernels go out with programmatic dependent launch: the prep kernel
+// waits inside for the previous kernel on the stream, the decode kernel's
+// producer for the prep kernel (see gemv.cuh).
 template <int M>
-tb_status launch_gemv(const LinearArgs& a, const DevInfo* d, const GemvPlan& pl, const GemvParams& p,
-                      bool fused) {
+tb_status launch_gemv(const LinearArgs& a, const DevInfo* d, const GemvPlan& pl, const CUtensorMap& tm,
+                      const GemvParams& p) {
   auto k = a.yt == TB_FP32 ? gemv_2bit_kernel<M, float> : gemv_2bit_kernel<M, __nv_bfloat16>;
   if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
-  if (fused) {
-    k<<<dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st>>>(p);
-    return launch_status();
-  }
-  return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, p);
+  return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, tm, p);
 }
 
 template <typename TIn>
@@ -326,31 +358,33 @@ tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
   GemvPlan pl;
   if (!gemv_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
   uint8_t* act = static_cast<uint8_t*>(a.ws);
-  const bool fused = a.M * (a.K / kHB) <= kGemvFusedMaxBlocks;
-  if (!fused) {
-    dim3 pgrid(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
-    prep_gemv_kernel<TIn><<<pgrid, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, act, a.K);
-    if (launch_status() != TB_OK) return TB_ERR_CUDA;
-  }
+  CUtensorMap tm;
+  if (make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.packed, a.K / 4, a.N, a.K / 4, 128,
+                  static_cast<uint32_t>(pl.R), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+    return TB_ERR_CUDA;
+  const dim3 pgrid(static_cast<unsigned>(a.K / kHB), static_cast<unsigned>(a.M));
+  if (launch_pdl(prep_gemv_kernel<TIn>, pgrid, dim3(kHThreads), 0, a.st, static_cast<const TIn*>(a.x), a.signs, act,
+                 static_cast<int>(a.K), pl.NB) != TB_OK)
+    return TB_ERR_CUDA;
   GemvParams p;
   p.act = act;
-  p.x = a.x;
-  p.signs = a.signs;
-  p.xt = a.xt == TB_BF16 ? 0 : (a.xt == TB_FP16 ? 1 : 2);
-  p.fused = fused ? 1 : 0;
-  p.packed = a.packed;
   p.scales = a.scales;
   p.y = a.y;
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
-  p.seg_rows = pl.seg_rows;
+  p.R = pl.R;
+  p.RT = pl.RT;
+  p.NB = pl.NB;
+  p.nstage = pl.nstage;
   p.nslots = pl.nslots;
-  p.max_rows = pl.max_rows;
+  p.box_stride = pl.box_stride;
+  p.slot_bytes = pl.slot_bytes;
+  p.sc_bytes = pl.sc_bytes;
   switch (static_cast<int>(a.M)) {
-    case 1: return launch_gemv<1>(a, d, pl, p, fused);
-    case 2: return launch_gemv<2>(a, d, pl, p, fused);
-    case 3: return launch_gemv<3>(a, d, pl, p, fused);
-    case 4: return launch_gemv<4>(a, d, pl, p, fused);
+    case 1: return launch_gemv<1>(a, d, pl, tm, p);
+    case 2: return launch_gemv<2>(a, d, pl, tm, p);
+    case 3: return launch_gemv<3>(a, d, pl, tm, p);
+    case 4: return launch_gemv<4>(a, d, pl, tm, p);
     default: return TB_ERR_SHAPE;
   }
 }
@@ -741,7 +775,7 @@ tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* p
   if (st != TB_OK) return st;
   if (xt == TB_INT8) return TB_ERR_DTYPE;
   if (M > kGemvMaxM || K % 1024 != 0) return TB_ERR_SHAPE;
-  const int64_t need = std::max<int64_t>(M * gemv_act_row_bytes(K), gtc_ws_bytes(M, K));
+  const int64_t need = gemv_ws_bytes(M, K);
   if (need > static_cast<int64_t>(TB_NOALLOC_SCRATCH_BYTES)) return TB_ERR_WORKSPACE;
   if (!aligned(packed, 16) || !aligned(scales, 16) || !aligned(x, 16) || !aligned(y, 16) ||
       (signs != nullptr && !aligned(signs, 16)))

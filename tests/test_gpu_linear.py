@@ -58,6 +58,10 @@ WORKLOAD_CASES = [
     (2, 4, 5120, 17408, 0.5, "lognormal", 0.0),
     (9, 3, 1001, 2048, 0.33, "abs_normal", 0.0),       # ragged N (not a multiple of 4)
     (8, 1, 4, 1024, 0.33, "abs_normal", 0.0),          # fewer rows than one quad
+    (10, 1, 20000, 1024, 0.33, "abs_normal", 0.0),     # more CTAs than SMs (rows per CTA capped)
+    (11, 2, 6144, 6144, 0.2, "abs_normal", 0.0),       # q-projection shape
+    (12, 1, 1024, 3072, 0.5, "abs_normal", 0.0),       # K/512 not a multiple of the stage width
+    (13, 3, 5120, 6144, 0.33, "abs_normal", 0.01),     # o-projection shape
 ]
 
 
@@ -251,7 +255,11 @@ def test_gemm_invalid_bytes_no_fault():
 GEMV_TC = tb.TB_PATH_GEMV_TC
 
 
-@pytest.mark.parametrize("case", WORKLOAD_CASES, ids=lambda c: f"m{c[1]}n{c[2]}k{c[3]}")
+# shapes within the tensor-core decode kernel's limit of 148 x 128 rows
+GEMV_TC_CASES = [c for c in WORKLOAD_CASES if c[2] <= 148 * 128]
+
+
+@pytest.mark.parametrize("case", GEMV_TC_CASES, ids=lambda c: f"m{c[1]}n{c[2]}k{c[3]}")
 def test_gemv_tensor_core_2bit(case):
     prob, ref = _problem(case[0], case[1], case[2], case[3], case[4], "2bit", case[5], case[6])
     _check(prob.linear(GEMV_TC), ref, prob.p)
