@@ -51,8 +51,9 @@ constexpr int kGemvMaxNB = 8;                       // boxes per stage at most
 constexpr int kGemvMaxSlots = 12;
 constexpr int kGemvSmemTarget = 227 * 1024;         // one CTA per SM
 
-// rows per CTA at most: 32 * kGemvMaxRowTiles(M)
-__host__ __device__ constexpr int gemv_max_row_tiles(int) { return 4; }
+constexpr int kGemvRowTiles = 4;  // rows per CTA <= 32 * kGemvRowTiles
+// rows per CTA at most: 32 * gemv_max_row_tiles(M)
+__host__ __device__ constexpr int gemv_max_row_tiles(int) { return kGemvRowTiles; }
 // codes per item
 __host__ __device__ constexpr int gemv_cpi(int M) { return M == 1 ? 128 : (M == 2 ? 64 : 32); }
 

@@ -15,6 +15,7 @@
 
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_b3.cuh"
 #include "gemv_tc.cuh"
 #include "hadamard.cuh"
 #include "pack.cuh"
@@ -203,6 +204,8 @@ size_t workspace_bytes(int64_t M, int64_t K) {
   if (g > b) b = g;
   const size_t v = static_cast<size_t>(gemv_ws_bytes(M, K));  // decode activation words
   if (v > b) b = v;
+  const size_t v3 = static_cast<size_t>(b3_ws_bytes(M, K));  // base-3 decode activation words
+  if (v3 > b) b = v3;
   return (b + 255) & ~static_cast<size_t>(255);
 }
 
@@ -266,6 +269,52 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, Gemv
   return true;
 }
 
+struct B3Plan {
+  int grid, R, RT, NB, nstage, nslots, box_stride, slot_bytes, sc_bytes;
+  size_t smem;
+};
+
+// Geometry of the base-3 decode kernel; false if these sizes do not fit it.
+bool b3_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, B3Plan* out) {
+  if (M < 1 || M > kGemvMaxM || K % 1024 != 0 || K < 1024 || N < 1 || sm_count < 1) return false;
+  B3Plan pl;
+  int64_t R = (N + sm_count - 1) / sm_count;
+  if (R > 32 * kGemvRowTiles) R = 32 * kGemvRowTiles;
+  pl.R = static_cast<int>(R);
+  pl.RT = static_cast<int>((R + 31) / 32);
+  pl.grid = static_cast<int>((N + R - 1) / R);
+  const int64_t G = K / 128, C = K / 1024;
+  int NB = 1;
+  while (NB < kGemvMaxNB && NB < C && static_cast<int64_t>(NB) * R * kB3BlockBytes < 12 * 1024) NB *= 2;
+  pl.NB = NB;
+  pl.nstage = static_cast<int>(b3_nstage(K, NB));
+  pl.box_stride = static_cast<int>(align_up(R * kB3BlockBytes, 1024));
+  pl.slot_bytes = static_cast<int>(align_up(static_cast<int64_t>(NB) * pl.box_stride +
+                                                b3_act_stage_bytes(static_cast<int>(M), NB), 1024));
+  pl.sc_bytes = static_cast<int>(align_up(R * G * 2, 1024));
+  if (R * G * 2 >= (int64_t(1) << 20)) return false;
+  const int64_t part = M * pl.RT * 32 * kGemvWarps * 4;
+  int64_t ns = (max_smem - b3_smem_bytes(pl.sc_bytes, 0, 0)) / pl.slot_bytes;
+  if (ns > kGemvMaxSlots) ns = kGemvMaxSlots;
+  if (ns >= pl.nstage) {
+    ns = pl.nstage;
+  } else {
+    // slots reused by warp groups taking alternate stages: nslots a multiple of Q
+    const int ips = NB * 8;
+    const int qg = ips >= kGemvWarps ? 1 : kGemvWarps / ips;
+    ns -= ns % qg;
+    if (ns < qg || ns < 2) return false;
+  }
+  while (ns * pl.slot_bytes < part && ns < kGemvMaxSlots) ++ns;
+  if (ns * pl.slot_bytes < part) return false;
+  pl.nslots = static_cast<int>(ns);
+  const int64_t smem = b3_smem_bytes(pl.sc_bytes, pl.slot_bytes, pl.nslots);
+  if (smem > max_smem) return false;
+  pl.smem = static_cast<size_t>(smem);
+  *out = pl;
+  return true;
+}
+
 struct GtcPlan {
   int grid, box_rows, rows_box, parts, gpp, nb, nstages, depth;
   uint32_t w_box_bytes, box_stride, part_bytes, stage_bytes, tmem_cols;
@@ -316,10 +365,15 @@ constexpr int kB200Sms = 148;
 constexpr int kB200SmemOptin = 232448;
 
 bool gemv_ok(const LinearArgs& a) {
+  if (!(is_float_dtype(a.xt) && a.M >= 1 && a.M <= kGemvMaxM && a.K % 1024 == 0 && fast_aligned(a) &&
+        a.N < (int64_t(1) << 30)))
+    return false;
+  if (a.f == TB_FMT_BASE3) {
+    B3Plan pl;
+    return b3_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
+  }
   GemvPlan pl;
-  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGemvMaxM &&
-         a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30) &&
-         gemv_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
+  return gemv_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
 }
 
 bool gemv_tc_ok(const LinearArgs& a) {
@@ -451,7 +505,59 @@ tb_status run_gemv_tc(const LinearArgs& a, const DevInfo* d) {
   }
 }
 
+template <int M>
+tb_status launch_b3(const LinearArgs& a, const DevInfo* d, const B3Plan& pl, const CUtensorMap& tm,
+                    const GemvB3Params& p) {
+  auto k = a.yt == TB_FP32 ? gemv_b3_kernel<M, float> : gemv_b3_kernel<M, __nv_bfloat16>;
+  if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
+  return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, tm, p);
+}
+
+template <typename TIn>
+tb_status run_b3_typed(const LinearArgs& a, const DevInfo* d) {
+  B3Plan pl;
+  if (!b3_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
+  uint8_t* act = static_cast<uint8_t*>(a.ws);
+  const int64_t row_bytes = (a.K / 128) * kB3GroupBytes;
+  CUtensorMap tm;
+  if (make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.packed, row_bytes, a.N, row_bytes, kB3BlockBytes,
+                  static_cast<uint32_t>(pl.R)) != TB_OK)
+    return TB_ERR_CUDA;
+  const dim3 pgrid(static_cast<unsigned>(a.K / kHB), static_cast<unsigned>(a.M));
+  if (launch_pdl(prep_b3_kernel<TIn>, pgrid, dim3(kHThreads), 0, a.st, static_cast<const TIn*>(a.x), a.signs, act,
+                 static_cast<int>(a.K), pl.NB) != TB_OK)
+    return TB_ERR_CUDA;
+  GemvB3Params p;
+  p.act = act;
+  p.scales = a.scales;
+  p.y = a.y;
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.R = pl.R;
+  p.RT = pl.RT;
+  p.NB = pl.NB;
+  p.nstage = pl.nstage;
+  p.nslots = pl.nslots;
+  p.box_stride = pl.box_stride;
+  p.slot_bytes = pl.slot_bytes;
+  p.sc_bytes = pl.sc_bytes;
+  switch (static_cast<int>(a.M)) {
+    case 1: return launch_b3<1>(a, d, pl, tm, p);
+    case 2: return launch_b3<2>(a, d, pl, tm, p);
+    case 3: return launch_b3<3>(a, d, pl, tm, p);
+    case 4: return launch_b3<4>(a, d, pl, tm, p);
+    default: return TB_ERR_SHAPE;
+  }
+}
+
 tb_status run_gemv(const LinearArgs& a, const DevInfo* d) {
+  if (a.f == TB_FMT_BASE3) {
+    switch (a.xt) {
+      case TB_BF16: return run_b3_typed<__nv_bfloat16>(a, d);
+      case TB_FP16: return run_b3_typed<__half>(a, d);
+      default: return run_b3_typed<float>(a, d);
+    }
+  }
   switch (a.xt) {
     case TB_BF16: return run_gemv_typed<__nv_bfloat16>(a, d);
     case TB_FP16: return run_gemv_typed<__half>(a, d);

@@ -72,6 +72,13 @@ def test_gemv_2bit(case):
     _check(y, ref, prob.p)
 
 
+@pytest.mark.parametrize("case", WORKLOAD_CASES, ids=lambda c: f"m{c[1]}n{c[2]}k{c[3]}")
+def test_gemv_base3(case):
+    prob, ref = _problem(*case[:5], "base3", *case[5:])
+    y = prob.linear(GEMV)
+    _check(y, ref, prob.p)
+
+
 @pytest.mark.parametrize("fmt", ["2bit", "base3"])
 @pytest.mark.parametrize("case", WORKLOAD_CASES[:3] + WORKLOAD_CASES[5:],
                          ids=lambda c: f"m{c[1]}n{c[2]}k{c[3]}")
@@ -94,17 +101,19 @@ def test_auto_path_matches_oracle(fmt):
     _check(prob.linear(AUTO), ref, prob.p)
 
 
+@pytest.mark.parametrize("fmt", ["2bit", "base3"])
 @pytest.mark.parametrize("path", [GEMV, SIMPLE])
-def test_bf16_output(path):
-    prob, ref = _problem(0, 1, 256, 1024, 1 / 3, "2bit")
+def test_bf16_output(path, fmt):
+    prob, ref = _problem(0, 1, 256, 1024, 1 / 3, fmt)
     y = prob.linear(path, yt=tb.TB_BF16)
     _check(y, ref, prob.p)
 
 
 @pytest.mark.parametrize("path", [GEMV, SIMPLE])
 @pytest.mark.parametrize("xt", [tb.TB_FP16, tb.TB_FP32])
-def test_other_input_dtypes(path, xt):
-    prob, ref = _problem(0, 2, 256, 1024, 1 / 3, "2bit")
+@pytest.mark.parametrize("fmt", ["2bit", "base3"])
+def test_other_input_dtypes(path, xt, fmt):
+    prob, ref = _problem(0, 2, 256, 1024, 1 / 3, fmt)
     xf = torch.from_numpy(prob.p.x).to(DEV)
     x = xf.to(torch.float16 if xt == tb.TB_FP16 else torch.float32)
     # bf16 values are exact in fp32; in fp16 they may round, so use fp16's own values
@@ -114,9 +123,10 @@ def test_other_input_dtypes(path, xt):
     _check(y, ref, prob.p)
 
 
+@pytest.mark.parametrize("fmt", ["2bit", "base3"])
 @pytest.mark.parametrize("path", [GEMV, SIMPLE])
-def test_prerotated_input_without_signs(path):
-    prob, ref = _problem(1, 1, 17408, 5120, 0.33, "2bit", "abs_normal", 0.01)
+def test_prerotated_input_without_signs(path, fmt):
+    prob, ref = _problem(1, 1, 17408, 5120, 0.33, fmt, "abs_normal", 0.01)
     xr = orc.rotate(prob.p.x, prob.p.signs)
     x = torch.from_numpy(xr.astype(np.float32)).to(DEV)
     y = prob.linear(path, x=x, xt=tb.TB_FP32, signs=None)
@@ -173,8 +183,9 @@ def test_integer_mode_bitexact(fmt, m, n, k):
     assert np.array_equal(y.cpu().numpy().astype(np.int64), orc.linear_int(x, codes))
 
 
-def test_invalid_packed_bytes_do_not_fault():
-    prob, _ = _problem(0, 1, 256, 1024, 1 / 3, "2bit")
+@pytest.mark.parametrize("fmt", ["2bit", "base3"])
+def test_invalid_packed_bytes_do_not_fault(fmt):
+    prob, _ = _problem(0, 1, 256, 1024, 1 / 3, fmt)
     bad = torch.full_like(prob.packed, 0xFF)
     for path in (GEMV, SIMPLE):
         y = prob.linear(path, packed=bad)
@@ -182,8 +193,9 @@ def test_invalid_packed_bytes_do_not_fault():
     assert tb.tb_get_device_fault() == 0
 
 
-def test_repeated_calls_are_deterministic_gemv():
-    prob, ref = _problem(2, 4, 5120, 17408, 0.5, "2bit", "lognormal", 0.0)
+@pytest.mark.parametrize("fmt", ["2bit", "base3"])
+def test_repeated_calls_are_deterministic_gemv(fmt):
+    prob, ref = _problem(2, 4, 5120, 17408, 0.5, fmt, "lognormal", 0.0)
     a = prob.linear(GEMV)
     b = prob.linear(GEMV)
     assert np.array_equal(a, b)
