@@ -23,8 +23,8 @@
 // Geometry: a box is one 1024-block of K, 208 bytes, of each of the CTA's R
 // rows (no swizzle; a row pitch of 13 16-byte chunks makes lane = row loads of
 // one chunk conflict-free).  A group starts at byte 26 g of the block, which
-// is 16-byte aligned only for g = 0, so the item code is instantiated per g
-// with the chunk loads and the 2-byte funnel shift fixed at compile time.
+// is 16-byte aligned only for g = 0: three chunk loads cover it, and its words
+// are aligned with warp-uniform selects and a 2-byte funnel shift.
 // Pipeline, slots, refill and the final fixed-order reduction are those of the
 // 2-bit kernel.
 #pragma once
@@ -112,29 +112,31 @@ __device__ __forceinline__ uint32_t b3_fifth(uint32_t w) {
   return (t >> 6) & 0x03030303u;
 }
 
-// The 7 words (26 bytes + 2 more, of the next group or zero) of group GP of a
-// 208-byte block row at `row` (16-byte aligned).
-template <int GP>
-__device__ __forceinline__ void b3_group_words(const uint8_t* row, uint32_t (&G)[7]) {
-  constexpr int o = 26 * GP, c0 = o / 16, r = o % 16, nc = (r + 26 + 15) / 16;
+// The 7 words of group gp (0..7) of a 208-byte block row at `row` (16-byte
+// aligned): bytes 0..25 of the group, then 2 more bytes (of the next group, or
+// past the row: only the fifth-digit lanes with zero activations see them).
+// Three 16-byte loads cover the group wherever it starts; the word offset
+// (0..3) and the 2-byte shift are uniform across the warp and applied with
+// selects and a funnel shift, so one code path serves all eight positions.
+__device__ __forceinline__ void b3_group_words(const uint8_t* row, int gp, uint32_t (&G)[7]) {
+  const int o = 26 * gp, c0 = o >> 4, q = (o & 15) >> 2;
+  const uint32_t sh = (o & 2) ? 16u : 0u;
   uint32_t u[12];
 #pragma unroll
-  for (int i = 0; i < 12; ++i) u[i] = 0u;  // words past the loaded chunks only feed bytes 26, 27
-#pragma unroll
-  for (int c = 0; c < nc; ++c) {
+  for (int c = 0; c < 3; ++c) {
     const uint4 v = reinterpret_cast<const uint4*>(row)[c0 + c];
     u[4 * c] = v.x;
     u[4 * c + 1] = v.y;
     u[4 * c + 2] = v.z;
     u[4 * c + 3] = v.w;
   }
+  uint32_t v[10], w[8];
 #pragma unroll
-  for (int k = 0; k < 7; ++k) {
-    if constexpr (r % 4 == 0)
-      G[k] = u[r / 4 + k];
-    else
-      G[k] = __funnelshift_r(u[r / 4 + k], u[r / 4 + k + 1], 16);
-  }
+  for (int i = 0; i < 10; ++i) v[i] = (q & 2) ? u[i + 2] : u[i];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = (q & 1) ? v[i + 1] : v[i];
+#pragma unroll
+  for (int k = 0; k < 7; ++k) G[k] = __funnelshift_r(w[k], w[k + 1], sh);
 }
 
 // Integer sums  sum_k c_k hi_k  and  sum_k c_k lo_k  of one group of one row:
@@ -144,7 +146,7 @@ __device__ __forceinline__ void b3_dot(const uint32_t (&G)[7], const uint32_t* A
   int hh[4] = {0, 0, 0, 0}, ll[4] = {0, 0, 0, 0};
 #pragma unroll
   for (int n = 0; n < 26; ++n) {
-    const uint32_t b = (G[n >> 2] >> (8 * (n & 3))) & 0xFFu;
+    const uint32_t b = __byte_perm(G[n >> 2], 0u, 0x4440u + (n & 3));
     const uint32_t c = lut_lane[b << 5];
     hh[n & 3] = dp4a_us(c, A[n], hh[n & 3]);
     ll[n & 3] = dp4a_us(c, A[kB3PlaneWords + n], ll[n & 3]);
@@ -189,8 +191,8 @@ __device__ __forceinline__ void b3_issue_stage(const CUtensorMap* tm, const Gemv
   if (act) bulk_load(slot + p.NB * p.box_stride, p.act + static_cast<int64_t>(s) * abytes, abytes, &full[slot_i]);
 }
 
-// One item: group GP of box `box`, for up to kGemvRowTiles tiles of 32 rows.
-template <int M, int GP>
+// One item: group gs & 7 of box `box`, for up to kGemvRowTiles tiles of 32 rows.
+template <int M>
 __device__ __forceinline__ void b3_item(const uint8_t* box, const uint8_t* act, const __half* sc, const int (&roff)[4],
                                         const int (&soff)[4], int RT, int NB, int gs, int g, const uint32_t* lut_lane,
                                         float (&acc)[M][4]) {
@@ -215,7 +217,7 @@ __device__ __forceinline__ void b3_item(const uint8_t* box, const uint8_t* act, 
   for (int t = 0; t < kGemvRowTiles; ++t) {
     if (t < RT) {
       uint32_t G[7];
-      b3_group_words<GP>(box + roff[t], G);
+      b3_group_words(box + roff[t], gs & 7, G);
       const float s_rg = __half2float(sc[soff[t] + g]);
 #pragma unroll
       for (int m = 0; m < M; ++m) {
@@ -321,16 +323,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       const int g = s * 8 * p.NB + it;  // global group
       if (g >= G) continue;
       const uint8_t* box = slot + (it >> 3) * p.box_stride;
-      switch (it & 7) {
-        case 0: b3_item<M, 0>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-        case 1: b3_item<M, 1>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-        case 2: b3_item<M, 2>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-        case 3: b3_item<M, 3>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-        case 4: b3_item<M, 4>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-        case 5: b3_item<M, 5>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-        case 6: b3_item<M, 6>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-        default: b3_item<M, 7>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc); break;
-      }
+      b3_item<M>(box, act, sc, roff, soff, p.RT, p.NB, it, g, lut_lane, acc);
     }
     __syncwarp();
     if (lane == 0) {

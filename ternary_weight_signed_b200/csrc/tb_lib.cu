@@ -288,7 +288,8 @@ bool b3_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, B3Plan
   while (NB < kGemvMaxNB && NB < C && static_cast<int64_t>(NB) * R * kB3BlockBytes < 12 * 1024) NB *= 2;
   pl.NB = NB;
   pl.nstage = static_cast<int>(b3_nstage(K, NB));
-  pl.box_stride = static_cast<int>(align_up(R * kB3BlockBytes, 1024));
+  // + 16: the group-word loads of the last row may read one chunk past it
+  pl.box_stride = static_cast<int>(align_up(R * kB3BlockBytes + 16, 1024));
   pl.slot_bytes = static_cast<int>(align_up(static_cast<int64_t>(NB) * pl.box_stride +
                                                 b3_act_stage_bytes(static_cast<int>(M), NB), 1024));
   pl.sc_bytes = static_cast<int>(align_up(R * G * 2, 1024));
