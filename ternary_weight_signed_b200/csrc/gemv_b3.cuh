@@ -139,15 +139,22 @@ __device__ __forceinline__ void b3_group_words(const uint8_t* row, int gp, uint3
   for (int k = 0; k < 7; ++k) G[k] = __funnelshift_r(w[k], w[k + 1], sh);
 }
 
+// Entry b of this lane's copy of the table: shared address lut_lane + 128 b.
+__device__ __forceinline__ uint32_t b3_lut(uint32_t lut_lane, uint32_t b) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(lut_lane + (b << 7)));
+  return v;
+}
+
 // Integer sums  sum_k c_k hi_k  and  sum_k c_k lo_k  of one group of one row:
 // codes from the words G, activation planes A (hi at 0, lo at kB3PlaneWords).
-__device__ __forceinline__ void b3_dot(const uint32_t (&G)[7], const uint32_t* A, const uint32_t* lut_lane, int& h,
+__device__ __forceinline__ void b3_dot(const uint32_t (&G)[7], const uint32_t* A, uint32_t lut_lane, int& h,
                                        int& l) {
   int hh[4] = {0, 0, 0, 0}, ll[4] = {0, 0, 0, 0};
 #pragma unroll
   for (int n = 0; n < 26; ++n) {
     const uint32_t b = __byte_perm(G[n >> 2], 0u, 0x4440u + (n & 3));
-    const uint32_t c = lut_lane[b << 5];
+    const uint32_t c = b3_lut(lut_lane, b);
     hh[n & 3] = dp4a_us(c, A[n], hh[n & 3]);
     ll[n & 3] = dp4a_us(c, A[kB3PlaneWords + n], ll[n & 3]);
   }
@@ -194,7 +201,7 @@ __device__ __forceinline__ void b3_issue_stage(const CUtensorMap* tm, const Gemv
 // One item: group gs & 7 of box `box`, for up to kGemvRowTiles tiles of 32 rows.
 template <int M>
 __device__ __forceinline__ void b3_item(const uint8_t* box, const uint8_t* act, const __half* sc, const int (&roff)[4],
-                                        const int (&soff)[4], int RT, int NB, int gs, int g, const uint32_t* lut_lane,
+                                        const int (&soff)[4], int RT, int NB, int gs, int g, uint32_t lut_lane,
                                         float (&acc)[M][4]) {
   float e[M];
   int qs[M];
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     roff[t] = min(32 * t + lane, p.R - 1) * kB3BlockBytes;
     soff[t] = min(32 * t + lane, nrows - 1) * G;
   }
-  const uint32_t* lut_lane = lut + lane;
+  const uint32_t lut_lane = smem_u32(lut) + 4u * static_cast<uint32_t>(lane);  // shared address
 
   const int it0 = IPS >= NW ? warp : warp % IPS;
   const int q = IPS >= NW ? 0 : warp / IPS;
