@@ -476,6 +476,36 @@ def oracle_sample(fmt, seconds):
             "sample": f"{reps} x oracle.linear on {rows} of 17408 rows (K=5120, M=1), {el:.1f} s"}
 
 
+def run_sweep(args, rank, world):
+    """Down-projection decode sweep (K=17408, N=5120, M in {1,2,4,8,16}, both
+    packings): device time per call and packed-weight GB/s of each cell, timed
+    like the headline line.  Printed as its own JSON line (not the bench line)."""
+    import torch
+
+    from ternary_weight_signed_b200 import binding as tb
+    from ternary_weight_signed_b200 import build as tbbuild
+    from ternary_weight_signed_b200 import inputs
+
+    tbbuild.build()
+    tb.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    peak, peak_kind = _peaks()
+    w = inputs.WORKLOADS["gemv_down_k17408_n5120"]
+    cells = []
+    for fmt in ("2bit", "base3"):
+        for m in w["ms"]:
+            res = measure_decode(args, tb, inputs, dev, stream, fmt, m, w["n"], w["k"], w["seed"], w["p0"],
+                                 w["scale_kind"], w["outlier_rate"], world, sample=False)
+            res.pop("problem")
+            e = _decode_entry(res, peak, peak_kind, world)
+            e.update({"format": fmt, "M": m, "tokens_per_s": round(m / (res["ms_per_step"] * 1e-3), 1)})
+            cells.append(e)
+            torch.cuda.empty_cache()
+    return {"sweep": "decode GEMV down K=17408 N=5120", "cells": cells}
+
+
 def run_reference(args, rank, world):
     """The CPU oracle, as it stands, on the same workload: every step is one
     oracle.linear call on a 1024-row sample of the 17408-row matrix (about
@@ -519,6 +549,7 @@ def main():
     ap.add_argument("--fmt", default="2bit", choices=["2bit", "base3"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
+    ap.add_argument("--sweep", action="store_true", help="print the down-projection decode sweep instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -533,6 +564,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     if args.impl == "reference":
         res = run_reference(args, rank, world)
+    elif args.sweep:
+        res = run_sweep(args, rank, world)
     else:
         res = run_ours(args, rank, world)
         if rank == 0:

@@ -42,21 +42,30 @@ constexpr int kGtcGroups = 4;  // step parities (groups of four unpack warps)
 constexpr int kGtcUnpackWarps = 4 * kGtcGroups;
 constexpr int kGtcThreads = 32 * (2 + kGtcUnpackWarps);
 constexpr int kGtcMaxParts = 7;
-constexpr int kGtcMaxM = 4;
+constexpr int kGtcMaxM = 16;
+// Activation rows of the B operand (hi and lo plane of each token, padded):
+// 16 up to 8 tokens, 32 up to 16; the MMA's N and the D columns per step.
+__host__ __device__ constexpr int gtc_atom_rows(int M) { return M <= 8 ? 16 : 32; }
+__host__ __device__ constexpr int gtc_atom_bytes(int M) { return gtc_atom_rows(M) * 128; }
+// Token capacity of the kernel instance that serves M tokens.
+__host__ __device__ constexpr int gtc_capacity(int M) { return M <= 4 ? 4 : (M <= 8 ? 8 : 16); }
 // kind::i8: D s32 (bits 4-5 = 2), A u8 (bits 7-9 = 0), B s8 (bits 10-12 = 1),
-// both K-major, N = 16 (N >> 3 at bits 17-22), M = 128 (M >> 4 at bits 24-28).
-constexpr uint32_t kGtcIdesc = (2u << 4) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
+// both K-major, N (N >> 3 at bits 17-22), M = 128 (M >> 4 at bits 24-28).
+__host__ __device__ constexpr uint32_t gtc_idesc(int n) {
+  return (2u << 4) | (1u << 10) | ((static_cast<uint32_t>(n) >> 3) << 17) | ((128u >> 4) << 24);
+}
 
-// Activation workspace of this path: G atoms of 16 rows x 128 bytes (row 2m =
-// hi plane of token m, 2m + 1 = lo plane; rows >= 2M zero), each atom in the
+// Activation workspace of this path: G atoms of gtc_atom_rows(M) rows x 128
+// bytes (row 2m = hi plane of token m, 2m + 1 = lo plane; rows >= 2M zero), each atom in the
 // UMMA K-major 128-byte-swizzled layout (16-byte chunk c of row r at
 // 16 (c ^ (r & 7)), 8-row groups 1 KB apart); inside each 16-code chunk byte
 // 4j + b holds code k = 4b + j, the order in which ((w >> 2j) & 0x03030303)
 // delivers the packed codes.  Then info[M][G] = {float e_g, int sum of q}.
-constexpr int kGtcAtomBytes = 2048;
-__host__ __device__ constexpr int64_t gtc_atoms_bytes(int64_t K) { return (K / 128) * kGtcAtomBytes; }
+__host__ __device__ constexpr int64_t gtc_atoms_bytes(int64_t M, int64_t K) {
+  return (K / 128) * gtc_atom_bytes(static_cast<int>(M));
+}
 __host__ __device__ constexpr int64_t gtc_ws_bytes(int64_t M, int64_t K) {
-  return gtc_atoms_bytes(K) + M * (K / 128) * 8;
+  return gtc_atoms_bytes(M, K) + M * (K / 128) * 8;
 }
 
 template <typename TIn>
@@ -90,7 +99,8 @@ __global__ void __launch_bounds__(kHThreads) prep_gemv_tc_kernel(const TIn* __re
   // chunk c = (t / 2) % 8 of the group, half h = t % 2 of the chunk
   const int gl = t >> 4, c = (t >> 1) & 7, h = t & 1;
   const int64_t g = static_cast<int64_t>(blk) * 8 + gl;
-  uint8_t* atom = ws + g * kGtcAtomBytes;
+  const int AR = gtc_atom_rows(M);
+  uint8_t* atom = ws + g * gtc_atom_bytes(M);
   uint8_t hb[16], lb[16];  // this thread's 8 bytes land in half of a 16-byte chunk
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -121,14 +131,14 @@ __global__ void __launch_bounds__(kHThreads) prep_gemv_tc_kernel(const TIn* __re
   const uint4 val = h ? make_uint4(wl[0], wl[1], wl[2], wl[3]) : make_uint4(wh[0], wh[1], wh[2], wh[3]);
   *reinterpret_cast<uint4*>(atom + row * 128 + 16 * (c ^ (row & 7))) = val;
   if (m == 0) {  // rows of tokens >= M are zero
-    for (int r = 2 * M + h; r < 16; r += 2)
+    for (int r = 2 * M + h; r < AR; r += 2)
       *reinterpret_cast<uint4*>(atom + r * 128 + 16 * (c ^ (r & 7))) = make_uint4(0, 0, 0, 0);
   }
   if ((t & 15) == 0) {
     int2 inf;
     inf.x = __float_as_int(e);
     inf.y = qs;
-    reinterpret_cast<int2*>(ws + gtc_atoms_bytes(K))[m * (K / 128) + g] = inf;
+    reinterpret_cast<int2*>(ws + gtc_atoms_bytes(M, K))[m * (K / 128) + g] = inf;
   }
 }
 
@@ -136,6 +146,7 @@ struct GemvTcParams {
   const uint8_t* act;      // prep_gemv_tc output
   const uint16_t* scales;  // [N, G] fp16 bits
   void* y;                 // [M, N]
+  int M;                   // tokens (<= the kernel's capacity MT)
   int N, K;
   int box_rows;            // rows of every TMA box (max rows of any CTA)
   int rows_box;            // TMEM lanes per part (box_rows rounded up to 32)
@@ -189,6 +200,19 @@ __device__ __forceinline__ void tmem_ld_cols<4>(uint32_t taddr, uint32_t (&r)[4]
                : "r"(taddr));
 }
 template <>
+__device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld_cols<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld32(taddr, r);
+}
+template <>
 __device__ __forceinline__ void tmem_ld_cols<8>(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
@@ -207,12 +231,16 @@ __host__ __device__ inline int64_t gtc_smem_bytes(int M, int64_t K, int box_rows
                                                   int nstages, int depth) {
   const int64_t G = K / 128;
   return 1024 + static_cast<int64_t>(nstages) * stage_bytes + align128(box_rows * G * 2) + align128(M * G * 8) +
-         align128(kGtcGroups * 128 * M * 4) + 8 * (2 * nstages + depth + 2) + 16;
+         align128(kGtcGroups * 128 * gtc_capacity(M) * 4) + 8 * (2 * nstages + depth + 2) + 16;
 }
 
-template <int M, typename TOut>
+template <int MT, typename TOut>
 __global__ void __launch_bounds__(kGtcThreads, 1)
     gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvTcParams p) {
+  constexpr int AR = gtc_atom_rows(MT);      // activation rows, MMA N, D columns per step
+  constexpr int ATOM = gtc_atom_bytes(MT);
+  constexpr uint32_t IDESC = gtc_idesc(AR);
+  const int M = p.M;
   // tm_w: the packed codes as uint32 [N rows][K/16], box 32 x box_rows, 128B swizzle
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -230,7 +258,7 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
   __half* sc = reinterpret_cast<__half*>(stages + static_cast<int64_t>(p.nstages) * p.stage_bytes);
   int2* info = reinterpret_cast<int2*>(reinterpret_cast<uint8_t*>(sc) + align128(p.box_rows * G * 2));
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(info) + align128(M * G * 8));
-  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + align128(kGtcGroups * 128 * M * 4));
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + align128(kGtcGroups * 128 * MT * 4));
   uint64_t* empty = full + p.nstages;
   uint64_t* d_ready = empty + p.nstages;
   uint64_t* sb_bar = d_ready + p.depth;  // scales + info
@@ -266,7 +294,7 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
       const uint32_t sbytes = static_cast<uint32_t>(nrows) * G * 2;
       mbar_arrive_expect_tx(sb_bar, sbytes + static_cast<uint32_t>(M * G * 8));
       bulk_load(sc, p.scales + static_cast<int64_t>(r0) * G, sbytes, sb_bar);
-      bulk_load(info, p.act + gtc_atoms_bytes(K), static_cast<uint32_t>(M * G * 8), sb_bar);
+      bulk_load(info, p.act + gtc_atoms_bytes(M, K), static_cast<uint32_t>(M * G * 8), sb_bar);
       const int bpp = p.gpp / 4;  // 512-code blocks per part
       for (int s = 0; s < nst; ++s) {
         const int slot = s % p.nstages;
@@ -277,7 +305,7 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
         for (int pt = 0; pt < p.parts; ++pt) {
           const int g0 = pt * p.gpp + s * gps;  // first group of this stage and part
           nat[pt] = max(0, min(gps, min(G - g0, p.gpp - s * gps)));
-          bytes += p.nb * p.w_box_bytes + static_cast<uint32_t>(nat[pt]) * kGtcAtomBytes;
+          bytes += p.nb * p.w_box_bytes + static_cast<uint32_t>(nat[pt]) * ATOM;
         }
         mbar_arrive_expect_tx(&full[slot], bytes);
         for (int pt = 0; pt < p.parts; ++pt) {
@@ -285,9 +313,9 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
           for (int b = 0; b < p.nb; ++b)
             tma_load_2d(pw + b * p.box_stride, &tm_w, (pt * bpp + s * p.nb + b) * 32, r0, &full[slot]);
           if (nat[pt] > 0)
-            bulk_load(pw + (p.part_bytes - gps * kGtcAtomBytes),
-                      p.act + static_cast<int64_t>(pt * p.gpp + s * gps) * kGtcAtomBytes,
-                      static_cast<uint32_t>(nat[pt]) * kGtcAtomBytes, &full[slot]);
+            bulk_load(pw + (p.part_bytes - gps * ATOM),
+                      p.act + static_cast<int64_t>(pt * p.gpp + s * gps) * ATOM,
+                      static_cast<uint32_t>(nat[pt]) * ATOM, &full[slot]);
         }
       }
     }
@@ -301,9 +329,9 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
     const int r = L - pt * p.rows_box;         // row (within the CTA) of this lane
     const bool live = pt < p.parts && r < nrows;
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-    float acc[M];
+    float acc[MT];
 #pragma unroll
-    for (int m = 0; m < M; ++m) acc[m] = 0.f;
+    for (int m = 0; m < MT; ++m) acc[m] = 0.f;
     // The other parts' columns of this lane stay zero for the whole kernel.
     if (p.parts > 1) {
       uint32_t z[32];
@@ -320,17 +348,19 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
       const int d = jj & dmask;
       ok = ok && mbar_wait(&d_ready[d], (jj >> p.depth_log2) & 1, FAULT_WAIT_MMA);
       tc_fence_after();
-      uint32_t dv[2 * M > 2 ? (2 * M > 4 ? 8 : 4) : 2];
-      tmem_ld_cols(tmem_d0 + 16u * d + lane_off, dv);
+      uint32_t dv[2 * MT];
+      tmem_ld_cols(tmem_d0 + static_cast<uint32_t>(AR) * d + lane_off, dv);
       tmem_ld_wait();
       const int g = pt * p.gpp + jj;
       if (live && g < G) {
         const float s = __half2float(sc[r * G + g]);
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const int2 inf = info[m * G + g];
-          const int v = static_cast<int>(dv[2 * m]) * 256 + static_cast<int>(dv[2 * m + 1]) - inf.y;
-          acc[m] = fmaf(__int2float_rn(v), s * __int_as_float(inf.x), acc[m]);
+        for (int m = 0; m < MT; ++m) {
+          if (m < M) {
+            const int2 inf = info[m * G + g];
+            const int v = static_cast<int>(dv[2 * m]) * 256 + static_cast<int>(dv[2 * m + 1]) - inf.y;
+            acc[m] = fmaf(__int2float_rn(v), s * __int_as_float(inf.x), acc[m]);
+          }
         }
       }
     };
@@ -378,11 +408,11 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
           for (int pp = 0; pp < p.parts; ++pp) {
             if (pp * p.gpp + j >= G) continue;  // this part has no group j
             const uint32_t b_atom = smem_u32(st + static_cast<int64_t>(pp) * p.part_bytes +
-                                             (p.part_bytes - gps * kGtcAtomBytes) + (j & gmask) * kGtcAtomBytes);
+                                             (p.part_bytes - gps * ATOM) + (j & gmask) * ATOM);
             const uint32_t a_col = tmem + static_cast<uint32_t>(d) * a_cols + 32u * pp;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              umma_i8_ts(tmem_d0 + 16u * d, a_col + 8u * kk, umma_desc_sw128(b_atom + 32u * kk), kGtcIdesc,
+              umma_i8_ts(tmem_d0 + static_cast<uint32_t>(AR) * d, a_col + 8u * kk, umma_desc_sw128(b_atom + 32u * kk), IDESC,
                          first_mma ? 0u : 1u);
               first_mma = false;
             }
@@ -399,7 +429,8 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
     // partial sums of the four groups of this lane, then the parts of each row
     float* rs = red + (sub * 128 + L) * M;
 #pragma unroll
-    for (int m = 0; m < M; ++m) rs[m] = live ? acc[m] : 0.f;
+    for (int m = 0; m < MT; ++m)
+      if (m < M) rs[m] = live ? acc[m] : 0.f;
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kGtcUnpackWarps) : "memory");
     TOut* y = reinterpret_cast<TOut*>(p.y);
     for (int i = threadIdx.x - 64; i < nrows * M; i += 32 * kGtcUnpackWarps) {

@@ -331,22 +331,23 @@ bool gtc_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, GtcPl
   if (pl.box_rows > 128) return false;
   pl.rows_box = 32 * ((pl.box_rows + 31) / 32);
   const int G = static_cast<int>(K / 128);
+  const int AR = gtc_atom_rows(static_cast<int>(M));  // D columns per step
   int parts = 128 / pl.rows_box;
-  if (parts > 3) parts = 3;  // TMEM: depth x (32 parts + 16) columns with depth >= 4
+  if (parts > 3) parts = 3;  // TMEM: depth x (32 parts + AR) columns with depth >= 4
   if (parts > G / 4) parts = G / 4;
   if (parts < 1) parts = 1;
   pl.gpp = 4 * ((G + 4 * parts - 1) / (4 * parts));
   pl.parts = (G + pl.gpp - 1) / pl.gpp;
   pl.depth = 8;  // a multiple of the 4 step groups
-  if (pl.depth * (32 * pl.parts + 16) > 512) pl.depth = 4;
-  const int cols = pl.depth * (32 * pl.parts + 16);
+  if (pl.depth * (32 * pl.parts + AR) > 512) pl.depth = 4;
+  const int cols = pl.depth * (32 * pl.parts + AR);
   if (cols > 512) return false;
   pl.tmem_cols = 32;
   while (static_cast<int>(pl.tmem_cols) < cols) pl.tmem_cols <<= 1;
   pl.w_box_bytes = static_cast<uint32_t>(pl.box_rows) * 128u;
   pl.box_stride = (pl.w_box_bytes + 1023u) & ~1023u;
   for (pl.nb = 2; pl.nb >= 1; --pl.nb) {
-    pl.part_bytes = pl.nb * pl.box_stride + 4u * pl.nb * kGtcAtomBytes;
+    pl.part_bytes = pl.nb * pl.box_stride + 4u * pl.nb * static_cast<uint32_t>(gtc_atom_bytes(static_cast<int>(M)));
     pl.stage_bytes = static_cast<uint32_t>(pl.parts) * pl.part_bytes;
     const int64_t fixed = gtc_smem_bytes(static_cast<int>(M), K, pl.box_rows, 0, 0, pl.depth) + 8 * 2 * 6;
     int64_t ns = (static_cast<int64_t>(max_smem) - fixed) / pl.stage_bytes;
@@ -365,13 +366,17 @@ bool gtc_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, GtcPl
 constexpr int kB200Sms = 148;
 constexpr int kB200SmemOptin = 232448;
 
+// Base-3 decode serves up to kB3MaxM tokens, in chunks of kGemvMaxM.
+constexpr int kB3MaxM = 16;
+
 bool gemv_ok(const LinearArgs& a) {
-  if (!(is_float_dtype(a.xt) && a.M >= 1 && a.M <= kGemvMaxM && a.K % 1024 == 0 && fast_aligned(a) &&
+  const int64_t maxm = a.f == TB_FMT_BASE3 ? kB3MaxM : kGemvMaxM;
+  if (!(is_float_dtype(a.xt) && a.M >= 1 && a.M <= maxm && a.K % 1024 == 0 && fast_aligned(a) &&
         a.N < (int64_t(1) << 30)))
     return false;
   if (a.f == TB_FMT_BASE3) {
     B3Plan pl;
-    return b3_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
+    return b3_plan(std::min<int64_t>(a.M, kGemvMaxM), a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
   }
   GemvPlan pl;
   return gemv_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
@@ -379,7 +384,7 @@ bool gemv_ok(const LinearArgs& a) {
 
 bool gemv_tc_ok(const LinearArgs& a) {
   GtcPlan pl;
-  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGemvMaxM &&
+  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGtcMaxM &&
          a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30) &&
          gtc_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
 }
@@ -391,7 +396,12 @@ bool gemm_ok(const LinearArgs& a) {
 
 int auto_path(const LinearArgs& a) {
   if (a.xt == TB_INT8) return TB_PATH_SIMPLE;
-  if (gemv_ok(a)) return TB_PATH_GEMV;
+  // 2-bit: the dp4a kernel's cost grows with M, the tensor-core one's hardly
+  // does; measured on B200 (K=17408, N=5120) the tensor-core kernel wins from
+  // 4 tokens on (31 us against 40 us).
+  if (a.f == TB_FMT_2BIT && a.M >= 4 && gemv_tc_ok(a)) return TB_PATH_GEMV_TC;
+  if (gemv_ok(a)) return TB_PATH_GEMV;       // M <= 4 (2-bit), M <= 16 (base-3)
+  if (gemv_tc_ok(a)) return TB_PATH_GEMV_TC;  // 2-bit, up to 16 tokens
   if (gemm_ok(a)) return TB_PATH_GEMM;
   return TB_PATH_SIMPLE;
 }
@@ -459,6 +469,7 @@ tb_status run_gemv_tc_typed(const LinearArgs& a, const DevInfo* d, const GtcPlan
   p.act = act;
   p.scales = a.scales;
   p.y = a.y;
+  p.M = static_cast<int>(a.M);
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
   p.box_rows = pl.box_rows;
@@ -486,11 +497,10 @@ tb_status run_gemv_tc_typed(const LinearArgs& a, const DevInfo* d, const GtcPlan
       if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                               \
       return launch_pdl(k, dim3(pl.grid), dim3(kGtcThreads), pl.smem, a.st, tm_w, p);  \
     }
-  switch (static_cast<int>(a.M)) {
-    TB_GTC_CASE(1)
-    TB_GTC_CASE(2)
-    TB_GTC_CASE(3)
+  switch (gtc_capacity(static_cast<int>(a.M))) {
     TB_GTC_CASE(4)
+    TB_GTC_CASE(8)
+    TB_GTC_CASE(16)
     default: return TB_ERR_SHAPE;
   }
 #undef TB_GTC_CASE
@@ -553,11 +563,21 @@ tb_status run_b3_typed(const LinearArgs& a, const DevInfo* d) {
 
 tb_status run_gemv(const LinearArgs& a, const DevInfo* d) {
   if (a.f == TB_FMT_BASE3) {
-    switch (a.xt) {
-      case TB_BF16: return run_b3_typed<__nv_bfloat16>(a, d);
-      case TB_FP16: return run_b3_typed<__half>(a, d);
-      default: return run_b3_typed<float>(a, d);
+    // more than kGemvMaxM tokens: one pass over the weights per chunk of tokens
+    for (int64_t m0 = 0; m0 < a.M; m0 += kGemvMaxM) {
+      LinearArgs c = a;
+      c.M = std::min<int64_t>(kGemvMaxM, a.M - m0);
+      c.x = static_cast<const uint8_t*>(a.x) + m0 * a.K * dtype_size(a.xt);
+      c.y = static_cast<uint8_t*>(a.y) + m0 * a.N * dtype_size(a.yt);
+      tb_status st;
+      switch (a.xt) {
+        case TB_BF16: st = run_b3_typed<__nv_bfloat16>(c, d); break;
+        case TB_FP16: st = run_b3_typed<__half>(c, d); break;
+        default: st = run_b3_typed<float>(c, d); break;
+      }
+      if (st != TB_OK) return st;
     }
+    return TB_OK;
   }
   switch (a.xt) {
     case TB_BF16: return run_gemv_typed<__nv_bfloat16>(a, d);

@@ -114,12 +114,17 @@ def test_linear_validation(lib):
 def test_path_selection(lib):
     p = tb.tb_ternary_linear_path
     assert p(tb.TB_BF16, "2bit", 1, 17408, 5120) == tb.TB_PATH_GEMV
-    assert p(tb.TB_BF16, "2bit", 4, 5120, 17408) == tb.TB_PATH_GEMV
+    assert p(tb.TB_BF16, "2bit", 3, 5120, 17408) == tb.TB_PATH_GEMV
+    assert p(tb.TB_BF16, "2bit", 4, 5120, 17408) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "2bit", 1, 256, 1152, has_signs=False) == tb.TB_PATH_SIMPLE
     assert p(tb.TB_BF16, "2bit", 1, 17408, 5120, aligned16=False) == tb.TB_PATH_SIMPLE
     assert p(tb.TB_INT8, "2bit", 4, 256, 1024, has_signs=False) == tb.TB_PATH_SIMPLE
     assert p(tb.TB_BF16, "2bit", 2048, 17408, 5120) == tb.TB_PATH_GEMM
-    assert p(tb.TB_BF16, "2bit", 5, 256, 1024) == tb.TB_PATH_GEMM
+    assert p(tb.TB_BF16, "2bit", 5, 256, 1024) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "2bit", 16, 5120, 17408) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "2bit", 17, 5120, 17408) == tb.TB_PATH_GEMM
+    assert p(tb.TB_BF16, "base3", 1, 17408, 5120) == tb.TB_PATH_GEMV
+    assert p(tb.TB_BF16, "base3", 16, 5120, 17408) == tb.TB_PATH_GEMV
     assert p(tb.TB_BF16, "base3", 2048, 17408, 5120) == tb.TB_PATH_SIMPLE
     assert p(tb.TB_BF16, "2bit", 1, 256, 1000) == -1
 

@@ -277,6 +277,20 @@ def test_gemv_tensor_core_2bit(case):
     _check(prob.linear(GEMV_TC), ref, prob.p)
 
 
+@pytest.mark.parametrize("m", [5, 8, 9, 16])
+def test_gemv_tensor_core_more_tokens(m):
+    """5..16 tokens: 16- and 32-row activation tiles (two planes per token)."""
+    prob, ref = _problem(25, m, 3001, 3072, 0.33, "2bit", "abs_normal", 0.01)
+    _check(prob.linear(GEMV_TC), ref, prob.p)
+
+
+@pytest.mark.parametrize("m", [5, 16])
+def test_gemv_base3_token_chunks(m):
+    """More than four tokens on base-3: one pass over the weights per chunk."""
+    prob, ref = _problem(26, m, 1001, 2048, 0.33, "base3")
+    _check(prob.linear(GEMV), ref, prob.p)
+
+
 def test_gemv_tensor_core_rejects_rows_beyond_tmem():
     """More rows than 148 CTAs x 128 TMEM lanes: the tensor-core decode kernel
     refuses the shape; the CUDA-core kernel takes it."""
