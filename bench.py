@@ -506,6 +506,103 @@ def run_sweep(args, rank, world):
     return {"sweep": "decode GEMV down K=17408 N=5120", "cells": cells}
 
 
+def run_stack(args, rank, world):
+    """The synthetic 27B-class layer stack: 64 layers x {q, k, v, o, gate, up,
+    down} of distinct ternary weights (5.8 GB in 2-bit slots, 4.8 GB in base-3),
+    M in {1, 4, 16, 64, 512} tokens, zero fraction in {0.2, 0.33, 0.5}, both
+    packings.  One pass = the 448 tb_ternary_linear calls of the stack, captured
+    in one CUDA graph; every linear reads its own synthetic input (no attention
+    or nonlinearity between them).  Reported per cell: device time per pass,
+    tokens/s = M / time, and packed-weight GB/s.  Printed as its own JSON line."""
+    import torch
+
+    from ternary_weight_signed_b200 import binding as tb
+    from ternary_weight_signed_b200 import build as tbbuild
+    from ternary_weight_signed_b200 import inputs
+
+    tbbuild.build()
+    tb.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    seed = 4
+    layers = args.stack_layers
+    shapes = inputs.STACK_LAYER_SHAPES
+    ms = [int(v) for v in args.stack_ms.split(",")]
+    p0s = [float(v) for v in args.stack_p0.split(",")]
+    fmts = args.stack_fmts.split(",")
+    peak, peak_kind = _peaks()
+    kdims = sorted({k for _, _, k in shapes})
+    xin = {}
+    for m in ms:
+        for k in kdims:
+            xb, sg = inputs.stack_activations(seed, m, k)
+            xin[(m, k)] = (torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16),
+                           torch.from_numpy(sg).to(dev))
+    cells = []
+    for p0 in p0s:
+        t_gen = time.perf_counter()
+        weights = {f: [] for f in fmts}
+        scales = []
+        for layer in range(layers):
+            for j, (_, n, k) in enumerate(shapes):
+                codes = inputs.stack_codes_torch(seed, layer, j, n, k, p0, dev)
+                for f in fmts:
+                    pk = torch.empty(tb.tb_packed_bytes(f, n, k), dtype=torch.uint8, device=dev)
+                    tb.tb_pack_ternary(f, codes, n, k, pk)
+                    weights[f].append(pk)
+                del codes
+                scales.append(torch.from_numpy(inputs.stack_scales(seed, layer, j, n, k).view(np.int16)).to(dev))
+        torch.cuda.synchronize()
+        t_gen = time.perf_counter() - t_gen
+        for f in fmts:
+            pass_bytes = sum(_packed_bytes(f, n, k) for _, n, k in shapes) * layers
+            for m in ms:
+                ys = {n: torch.empty(m, n, dtype=torch.float32, device=dev) for n in {n for _, n, _ in shapes}}
+                wsb = max(tb.tb_ternary_linear_workspace(f, m, n, k) for _, n, k in shapes)
+                ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+                sh = stream.cuda_stream
+                paths = sorted({tb.tb_ternary_linear_path(tb.TB_BF16, f, m, n, k, True, True) for _, n, k in shapes})
+
+                def one_pass():
+                    for layer in range(layers):
+                        for j, (_, n, k) in enumerate(shapes):
+                            x, sg = xin[(m, k)]
+                            idx = layer * len(shapes) + j
+                            tb.tb_ternary_linear(x, tb.TB_BF16, weights[f][idx], scales[idx], f, m, n, k, sg, ys[n],
+                                                 tb.TB_FP32, ws, wsb, stream=sh)
+
+                with torch.cuda.stream(stream):
+                    one_pass()
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        one_pass()
+                    g.replay()
+                stream.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                reps = 3
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    e1.record(stream)
+                e1.synchronize()
+                ms_pass = e0.elapsed_time(e1) / reps
+                gbs = pass_bytes / (ms_pass * 1e-3) / 1e9
+                cells.append({"format": f, "p0": p0, "M": m, "ms_per_pass": round(ms_pass, 4),
+                              "tokens_per_s": round(m / (ms_pass * 1e-3), 1), "weight_GBs": round(gbs, 1),
+                              "hbm_frac": round(gbs / peak, 4), "paths": paths,
+                              "calls_per_pass": layers * len(shapes)})
+                del g, ws, ys
+                torch.cuda.empty_cache()
+        del weights, scales
+        torch.cuda.empty_cache()
+    return {"stack": f"synthetic 27B-class layer stack, {layers} layers x {len(shapes)} linears",
+            "bytes_per_pass": {f: sum(_packed_bytes(f, n, k) for _, n, k in shapes) * layers for f in fmts},
+            "peak_GBs": peak, "peak_source": peak_kind, "cells": cells}
+
+
 def run_reference(args, rank, world):
     """The CPU oracle, as it stands, on the same workload: every step is one
     oracle.linear call on a 1024-row sample of the 17408-row matrix (about
@@ -550,6 +647,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--sweep", action="store_true", help="print the down-projection decode sweep instead")
+    ap.add_argument("--stack", action="store_true", help="print the 64-layer stack sweep instead")
+    ap.add_argument("--stack-layers", type=int, default=64)
+    ap.add_argument("--stack-ms", default="1,4,16,64,512")
+    ap.add_argument("--stack-p0", default="0.2,0.33,0.5")
+    ap.add_argument("--stack-fmts", default="2bit,base3")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -566,6 +668,8 @@ def main():
         res = run_reference(args, rank, world)
     elif args.sweep:
         res = run_sweep(args, rank, world)
+    elif args.stack:
+        res = run_stack(args, rank, world)
     else:
         res = run_ours(args, rank, world)
         if rank == 0:

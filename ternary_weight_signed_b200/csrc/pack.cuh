@@ -129,4 +129,40 @@ __global__ void unpack_base3_kernel(const uint16_t* __restrict__ in, int4* __res
   count_invalid(bad, counter);
 }
 
+// Base-3 groups (26 bytes) -> 2-bit slot groups (32 bytes), one thread per
+// group: the prefill GEMM consumes the 2-bit layout, so a base-3 matrix is
+// re-encoded into the caller's workspace first.  Invalid bytes decode as t = 0
+// (as tb_unpack_ternary does; the linear paths leave their output unspecified).
+__global__ void transcode_b3_to_2bit_kernel(const uint16_t* __restrict__ in, uint4* __restrict__ out,
+                                            int64_t ngroups) {
+  const int64_t gi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (gi >= ngroups) return;
+  const uint16_t* p = in + gi * 13;
+  uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int h = 0; h < 13; ++h) {
+    const uint32_t pair = p[h];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int byte_idx = 2 * h + e;
+      const uint32_t raw = (pair >> (8 * e)) & 0xffu;
+      uint32_t v = raw, dig[5];
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        dig[j] = v % 3u;
+        v /= 3u;
+      }
+      bool invalid = raw >= 243u;
+      if (byte_idx == 25) invalid = invalid || dig[3] != 1u || dig[4] != 1u;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        const int k = 5 * byte_idx + j;  // code index in the group
+        if (k < 128) w[k >> 4] |= (invalid ? 1u : dig[j]) << (2 * (k & 15));
+      }
+    }
+  }
+  out[2 * gi] = make_uint4(w[0], w[1], w[2], w[3]);
+  out[2 * gi + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 }  // namespace tb

@@ -198,6 +198,13 @@ struct LinearArgs {
   cudaStream_t st;
 };
 
+// Base-3 prefill (more than 16 tokens) re-encodes the weights to 2-bit slots
+// in the workspace, in front of the GEMM's own activations.
+size_t b3_transcode_bytes(int f, int64_t M, int64_t N, int64_t K) {
+  if (f != TB_FMT_BASE3 || M <= 16) return 0;
+  return (static_cast<size_t>(N) * static_cast<size_t>(K / 4) + 255) & ~static_cast<size_t>(255);
+}
+
 size_t workspace_bytes(int64_t M, int64_t K) {
   size_t b = static_cast<size_t>(4) * static_cast<size_t>(M) * static_cast<size_t>(K);
   const size_t g = static_cast<size_t>(gtc_ws_bytes(M, K));  // tensor-core decode activations
@@ -390,7 +397,9 @@ bool gemv_tc_ok(const LinearArgs& a) {
 }
 
 bool gemm_ok(const LinearArgs& a) {
-  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.K % 1024 == 0 && fast_aligned(a) &&
+  // base-3 is served by re-encoding to 2-bit slots first (more than 16 tokens)
+  if (a.f == TB_FMT_BASE3 && a.M <= 16) return false;
+  return is_float_dtype(a.xt) && a.K % 1024 == 0 && fast_aligned(a) &&
          (a.M + kGemmBM - 1) / kGemmBM <= 65535 && a.N < (int64_t(1) << 30);
 }
 
@@ -651,7 +660,24 @@ void launch_prep_gemm(const LinearArgs& a, __half* xh) {
   prep_gemm_kernel<TIn><<<pg, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, xh, a.K);
 }
 
+tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d);
+
 tb_status run_gemm(const LinearArgs& a, const DevInfo* d) {
+  if (a.f != TB_FMT_BASE3) return run_gemm_2bit(a, d);
+  const size_t tb = b3_transcode_bytes(a.f, a.M, a.N, a.K);
+  const int64_t ngroups = a.N * (a.K / 128);
+  transcode_b3_to_2bit_kernel<<<static_cast<unsigned>((ngroups + 255) / 256), 256, 0, a.st>>>(
+      reinterpret_cast<const uint16_t*>(a.packed), static_cast<uint4*>(a.ws), ngroups);
+  if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  LinearArgs c = a;
+  c.f = TB_FMT_2BIT;
+  c.packed = static_cast<const uint8_t*>(a.ws);
+  c.ws = static_cast<uint8_t*>(a.ws) + tb;
+  c.ws_bytes = a.ws_bytes - tb;
+  return run_gemm_2bit(c, d);
+}
+
+tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   __half* xh = static_cast<__half*>(a.ws);
   switch (a.xt) {
     case TB_BF16: launch_prep_gemm<__nv_bfloat16>(a, xh); break;
@@ -706,7 +732,8 @@ tb_status validate_linear(const LinearArgs& a) {
   if (a.signs != nullptr && !aligned(a.signs, 8)) return TB_ERR_ALIGN;
   if (a.f == TB_FMT_BASE3 && !aligned(a.packed, 2)) return TB_ERR_ALIGN;
   if (!int_mode) {
-    if (a.ws == nullptr || a.ws_bytes < workspace_bytes(a.M, a.K)) return TB_ERR_WORKSPACE;
+    if (a.ws == nullptr || a.ws_bytes < workspace_bytes(a.M, a.K) + b3_transcode_bytes(a.f, a.M, a.N, a.K))
+      return TB_ERR_WORKSPACE;
     if (!aligned(a.ws, 16)) return TB_ERR_ALIGN;
   }
   return TB_OK;
@@ -830,7 +857,7 @@ tb_status tb_hadamard_rotate(const void* x, tb_dtype xt, void* y, tb_dtype yt, c
 
 size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K) {
   if ((f != TB_FMT_2BIT && f != TB_FMT_BASE3) || M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
-  return workspace_bytes(M, K);
+  return workspace_bytes(M, K) + b3_transcode_bytes(f, M, N, K);
 }
 
 tb_status tb_ternary_linear_ex(const void* x, tb_dtype xt, const uint8_t* packed, const uint16_t* scales,
@@ -856,8 +883,8 @@ int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64
                reinterpret_cast<const uint16_t*>(base), f, M, N, K,
                has_signs ? reinterpret_cast<const int8_t*>(0x2000) : nullptr,
                reinterpret_cast<void*>(0x3000), xt == TB_INT8 ? TB_INT32 : TB_FP32,
-               reinterpret_cast<void*>(0x4000), workspace_bytes(M > 0 ? M : 1, K > 0 ? K : 128),
-               nullptr};
+               reinterpret_cast<void*>(0x4000),
+               workspace_bytes(M > 0 ? M : 1, K > 0 ? K : 128) + b3_transcode_bytes(f, M, N, K), nullptr};
   if (validate_linear(a) != TB_OK) return -1;
   return auto_path(a);
 }

@@ -158,3 +158,110 @@ def workload_inputs(name: str, m: int | None = None) -> LinearInputs:
     mm = w["ms"][0] if m is None else m
     return make_linear_inputs(w["seed"], mm, w["n"], w["k"], w["p0"], w["scale_kind"],
                               w["outlier_rate"])
+
+
+# ---------------------------------------------------------------------------
+# The synthetic layer stack: 64 layers x 7 matrices, 21.8 G ternary codes, too
+# many to draw on the host, so its codes come from a counter-based generator
+# that the device (torch) and the host (numpy) evaluate identically: code
+# (n, k) of matrix `mat` of layer `layer` is a function of its index alone.
+#
+# Generator: SplitMix64 (Steele, Lea and Flood, "Fast splittable pseudorandom
+# number generators", OOPSLA 2014): with a 64-bit state s and the counter i,
+#   z = s + (i + 1) * 0x9E3779B97F4A7C15
+#   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9
+#   z = (z ^ (z >> 27)) * 0x94D049BB133111EB
+#   out = z ^ (z >> 31)                         (all mod 2^64, logical shifts)
+# u = (out >> 11) * 2^-53 is uniform in [0, 1) and becomes a code with the
+# same thresholds as draw_codes.  The state of a matrix is the SplitMix64
+# output for counter 0 of the state seed * 2^20 + layer * 16 + mat.  Scales,
+# activations and signs of the stack are small and come from numpy's default
+# generator seeded with (seed, layer, mat) (stack_scales, stack_activations).
+
+_SM_GOLDEN = 0x9E3779B97F4A7C15
+_SM_M1 = 0xBF58476D1CE4E5B9
+_SM_M2 = 0x94D049BB133111EB
+_U64 = (1 << 64) - 1
+
+
+def _splitmix64_py(state: int, i: int) -> int:
+    z = (state + (i + 1) * _SM_GOLDEN) & _U64
+    z = ((z ^ (z >> 30)) * _SM_M1) & _U64
+    z = ((z ^ (z >> 27)) * _SM_M2) & _U64
+    return z ^ (z >> 31)
+
+
+def stack_state(seed: int, layer: int, mat: int) -> int:
+    """64-bit generator state of one matrix of the stack."""
+    return _splitmix64_py((seed << 20) + layer * 16 + mat, 0)
+
+
+def _codes_from_uniform_bits(top53, p0: float, xp):
+    lo = (1.0 - p0) / 2.0
+    mid = lo + p0
+    u = top53.astype(xp.float64) * (1.0 / 9007199254740992.0)
+    out = xp.ones(u.shape, dtype=xp.int8)
+    out[u < mid] = 0
+    out[u < lo] = -1
+    return out
+
+
+def stack_codes_rows_np(seed: int, layer: int, mat: int, rows, k: int, p0: float) -> np.ndarray:
+    """Codes of the given rows (any order) of one stack matrix, [len(rows), k] int8 (host)."""
+    rows = np.asarray(rows, dtype=np.uint64)
+    s = np.uint64(stack_state(seed, layer, mat))
+    i = rows[:, None] * np.uint64(k) + np.arange(k, dtype=np.uint64)[None, :]
+    with np.errstate(over="ignore"):
+        z = s + (i + np.uint64(1)) * np.uint64(_SM_GOLDEN)
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(_SM_M1)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(_SM_M2)
+        z = z ^ (z >> np.uint64(31))
+    return _codes_from_uniform_bits(z >> np.uint64(11), p0, np)
+
+
+def _i64(c: int) -> int:
+    """A 64-bit constant as the signed value with the same bits."""
+    return c - (1 << 64) if c >= (1 << 63) else c
+
+
+def stack_codes_torch(seed: int, layer: int, mat: int, n: int, k: int, p0: float, device,
+                      rows_per_chunk: int = 1024):
+    """All codes of one stack matrix, [n, k] int8, computed on `device` with torch
+    int64 arithmetic (wrap-around products, logical shifts by masking)."""
+    import torch
+
+    s = _i64(stack_state(seed, layer, mat))
+    out = torch.empty((n, k), dtype=torch.int8, device=device)
+    col = torch.arange(k, dtype=torch.int64, device=device)
+
+    def lsr(z, sh):
+        return (z >> sh) & ((1 << (64 - sh)) - 1)
+
+    lo = (1.0 - p0) / 2.0
+    mid = lo + p0
+    for r0 in range(0, n, rows_per_chunk):
+        r1 = min(n, r0 + rows_per_chunk)
+        i = torch.arange(r0, r1, dtype=torch.int64, device=device)[:, None] * k + col[None, :]
+        z = s + (i + 1) * _i64(_SM_GOLDEN)
+        z = (z ^ lsr(z, 30)) * _i64(_SM_M1)
+        z = (z ^ lsr(z, 27)) * _i64(_SM_M2)
+        z = z ^ lsr(z, 31)
+        u = lsr(z, 11).to(torch.float64) * (1.0 / 9007199254740992.0)
+        seg = torch.ones_like(u, dtype=torch.int8)
+        seg[u < mid] = 0
+        seg[u < lo] = -1
+        out[r0:r1] = seg
+    return out
+
+
+def stack_scales(seed: int, layer: int, mat: int, n: int, k: int) -> np.ndarray:
+    """fp16 g128 scales of one stack matrix, |N(0,1)| * 0.02."""
+    rng = np.random.default_rng([seed, layer, mat, 1])
+    return draw_scales(rng, n, k, "abs_normal")
+
+
+def stack_activations(seed: int, m: int, k: int) -> tuple[np.ndarray, np.ndarray]:
+    """bf16 activations [m, k] (bits) and +-1 signs [k] for the stack's inputs
+    of width k (one per input width; the linears' inputs are independent)."""
+    rng = np.random.default_rng([seed, k, m, 2])
+    return draw_activations(rng, m, k), draw_signs(rng, k)

@@ -125,7 +125,8 @@ def test_path_selection(lib):
     assert p(tb.TB_BF16, "2bit", 17, 5120, 17408) == tb.TB_PATH_GEMM
     assert p(tb.TB_BF16, "base3", 1, 17408, 5120) == tb.TB_PATH_GEMV
     assert p(tb.TB_BF16, "base3", 16, 5120, 17408) == tb.TB_PATH_GEMV
-    assert p(tb.TB_BF16, "base3", 2048, 17408, 5120) == tb.TB_PATH_SIMPLE
+    assert p(tb.TB_BF16, "base3", 17, 5120, 17408) == tb.TB_PATH_GEMM
+    assert p(tb.TB_BF16, "base3", 2048, 17408, 5120) == tb.TB_PATH_GEMM
     assert p(tb.TB_BF16, "2bit", 1, 256, 1000) == -1
 
 

@@ -219,6 +219,15 @@ def test_gemm_2bit(case):
     _check(prob.linear(GEMM), ref, prob.p)
 
 
+@pytest.mark.parametrize("m", [17, 300])
+def test_gemm_base3_via_reencoding(m):
+    """Base-3 prefill: the weights are re-encoded to 2-bit slots in the
+    workspace, then the tensor-core GEMM runs on them."""
+    prob, ref = _problem(27, m, 1001, 2048, 0.33, "base3", "abs_normal", 0.01)
+    _check(prob.linear(GEMM), ref, prob.p)
+    _check(prob.linear(AUTO), ref, prob.p)
+
+
 @pytest.mark.parametrize("yt", [tb.TB_FP32, tb.TB_BF16])
 @pytest.mark.parametrize("xt", [tb.TB_FP16, tb.TB_FP32])
 def test_gemm_dtypes(yt, xt):
