@@ -417,4 +417,169 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode at M = 1 with dynamic item distribution.  Same data path as
+// gemv_2bit_kernel<1> (boxes, slots, activation blocks, mask-mode dp4a), but
+// the warps take items (stage, group) in order from a CTA-wide counter, so a
+// warp that the issue scheduler serves more often simply takes more items and
+// all warps finish together.  Each item's row sums go to a partial buffer
+// indexed by the item, and the final sum over items runs in item order, so the
+// result does not depend on which warp took which item (bitwise
+// reproducible).  Every stage has its own full barrier (used once), so a warp
+// may wait for any stage; the warp completing the last item of stage s refills
+// its slot with stage s + nslots.
+__host__ __device__ inline int64_t gemv_dyn_part_bytes(int nstage, int NB, int RT) {
+  return align128(static_cast<int64_t>(nstage) * NB * 4 * RT * 32 * 4);
+}
+__host__ __device__ inline int64_t gemv_dyn_smem_bytes(int64_t sc_bytes, int64_t slot_bytes, int nslots, int nstage,
+                                                       int NB, int RT) {
+  return 1024 + sc_bytes + slot_bytes * nslots + gemv_dyn_part_bytes(nstage, NB, RT) + 8 * (nstage + 1) +
+         4 * (nstage + 2);
+}
+
+__device__ __forceinline__ void gemv_issue_stage_bar(const CUtensorMap* tm, const GemvParams& p, uint8_t* ring,
+                                                     uint64_t* bar, int s, int slot_i, int r0, uint32_t wbytes,
+                                                     uint32_t abytes, bool weights, bool act) {
+  uint8_t* slot = ring + static_cast<int64_t>(slot_i) * p.slot_bytes;
+  if (weights) {
+    mbar_arrive_expect_tx(bar, wbytes + abytes);
+    for (int b = 0; b < p.NB; ++b) tma_load_2d(slot + b * p.box_stride, tm, (s * p.NB + b) * 128, r0, bar);
+  }
+  if (act) bulk_load(slot + p.NB * p.box_stride, p.act + static_cast<int64_t>(s) * abytes, abytes, bar);
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    gemv_2bit_dyn_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
+  constexpr int RTM = kGemvRowTiles;
+  pdl_launch_dependents();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const __half* sc = reinterpret_cast<const __half*>(base);
+  uint8_t* ring = base + p.sc_bytes;
+  float* part = reinterpret_cast<float*>(ring + p.nslots * p.slot_bytes);
+  const int IPS = p.NB * 4;  // items (groups) per stage
+  const int nitems = p.nstage * IPS;
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(part) +
+                                               gemv_dyn_part_bytes(p.nstage, p.NB, p.RT));
+  uint64_t* sc_bar = full + p.nstage;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(sc_bar + 1);  // [0] next item, [1 + s] items done of stage s
+
+  const int G = p.K / 128;
+  const int r0 = blockIdx.x * p.R;
+  const int nrows = min(p.R, p.N - r0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t wbytes = static_cast<uint32_t>(p.NB) * static_cast<uint32_t>(p.R) * 128u;
+  const uint32_t abytes = static_cast<uint32_t>(gemv_act_stage_bytes(1, p.NB));
+  const int act_off = p.NB * p.box_stride;
+  const int pre = min(p.nslots, p.nstage);
+  const int RS = p.RT * 32;  // partial floats per item
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.nstage; ++s) {
+      mbar_init(&full[s], 1);
+      cnt[1 + s] = 0;
+    }
+    cnt[0] = 0;
+    mbar_init(sc_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tm_w);
+    const uint32_t sbytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(G * 2);
+    mbar_arrive_expect_tx(sc_bar, sbytes);
+    bulk_load(base, p.scales + static_cast<int64_t>(r0) * G, sbytes, sc_bar);
+    for (int s = 0; s < pre; ++s) gemv_issue_stage_bar(&tm_w, p, ring, &full[s], s, s, r0, wbytes, abytes, true, false);
+    pdl_wait();  // the prep kernel's activation blocks
+    for (int s = 0; s < pre; ++s) gemv_issue_stage_bar(&tm_w, p, ring, &full[s], s, s, r0, wbytes, abytes, false, true);
+  }
+  __syncthreads();
+
+  int roff[RTM], soff[RTM];
+#pragma unroll
+  for (int t = 0; t < RTM; ++t) {
+    roff[t] = min(32 * t + lane, p.R - 1) * 128;
+    soff[t] = min(32 * t + lane, nrows - 1) * G;
+  }
+  const int sw = lane & 7;
+  bool ok = mbar_wait_backoff(sc_bar, 0, FAULT_WAIT_ACT);
+  while (ok) {
+    int i = 0;
+    if (lane == 0) i = static_cast<int>(atomicAdd(&cnt[0], 1u));
+    i = __shfl_sync(0xffffffffu, i, 0);
+    if (i >= nitems) break;
+    const int s = i / IPS, it = i - s * IPS;
+    const int slot_i = s % p.nslots;
+    if (!mbar_wait_backoff(&full[s], 0, FAULT_WAIT_FULL)) {
+      ok = false;
+      break;
+    }
+    const uint8_t* slot = ring + slot_i * p.slot_bytes;
+    const int g = s * 4 * p.NB + it;
+    float a[RTM];
+#pragma unroll
+    for (int t = 0; t < RTM; ++t) a[t] = 0.f;
+    if (g < G) {
+      const uint8_t* act = slot + act_off;
+      uint32_t A[64];
+      const uint4* src = reinterpret_cast<const uint4*>(act + it * kGemvGroupBytes);
+#pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        const uint4 u4 = src[v];
+        A[4 * v] = u4.x; A[4 * v + 1] = u4.y; A[4 * v + 2] = u4.z; A[4 * v + 3] = u4.w;
+      }
+      const int2 inf = reinterpret_cast<const int2*>(act + 4 * p.NB * kGemvGroupBytes)[it];
+      const float e = __int_as_float(inf.x);
+      const uint8_t* box = slot + (it >> 2) * p.box_stride;
+      const int gl = it & 3;
+      const int c0 = ((2 * gl) ^ sw) << 4, c1 = ((2 * gl + 1) ^ sw) << 4;
+#pragma unroll
+      for (int t = 0; t < RTM; ++t) {
+        if (t < p.RT) {
+          const uint8_t* rp = box + roff[t];
+          const uint4 u0 = *reinterpret_cast<const uint4*>(rp + c0);
+          const uint4 u1 = *reinterpret_cast<const uint4*>(rp + c1);
+          const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          const float s_rg = __half2float(sc[soff[t] + g]);
+          a[t] = __int2float_rn(gemv_item_mask(w, A) - inf.y) * (s_rg * e);
+        }
+      }
+    }
+    float* pp = part + static_cast<int64_t>(i) * RS;
+#pragma unroll
+    for (int t = 0; t < RTM; ++t)
+      if (t < p.RT) pp[32 * t + lane] = a[t];
+    // the warp finishing the last item of stage s refills its slot
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&cnt[1 + s], 1u) == static_cast<uint32_t>(IPS - 1) && s + p.nslots < p.nstage) {
+        __threadfence_block();
+        gemv_issue_stage_bar(&tm_w, p, ring, &full[s + p.nslots], s + p.nslots, slot_i, r0, wbytes, abytes, true,
+                             true);
+      }
+    }
+  }
+  // every copy must have landed before the CTA exits
+  if (threadIdx.x == 0) {
+    for (int s = max(0, p.nstage - p.nslots); s < p.nstage; ++s)
+      if (!mbar_wait(&full[s], 0, FAULT_WAIT_FULL)) break;
+  }
+  __syncthreads();
+  // row r: four threads take the items i = 4 j + u (u = 0..3) and add them in
+  // order of j; their four sums are then added in order of u
+  TOut* y = reinterpret_cast<TOut*>(p.y);
+  for (int base_r = 0; base_r < nrows; base_r += kGemvThreads / 4) {
+    const int r = base_r + (threadIdx.x >> 2), u = threadIdx.x & 3;
+    float sum = 0.f;
+    if (r < nrows)
+      for (int it = u; it < nitems; it += 4) sum += part[static_cast<int64_t>(it) * RS + r];
+    const float s1 = __shfl_down_sync(0xffffffffu, sum, 1);
+    const float s2 = __shfl_down_sync(0xffffffffu, sum, 2);
+    const float s3 = __shfl_down_sync(0xffffffffu, sum, 3);
+    if (u == 0 && r < nrows) y[r0 + r] = from_f32<TOut>(((sum + s1) + s2) + s3);
+  }
+}
+
 }  // namespace tb

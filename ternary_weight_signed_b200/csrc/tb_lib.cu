@@ -454,6 +454,22 @@ tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
   p.box_stride = pl.box_stride;
   p.slot_bytes = pl.slot_bytes;
   p.sc_bytes = pl.sc_bytes;
+  if (a.M == 1) {
+    // dynamic item distribution: its own slot count (no warp-group constraint)
+    // and a partial-sum buffer of one float per item and row
+    const int64_t fixed = gemv_dyn_smem_bytes(pl.sc_bytes, 0, 0, pl.nstage, pl.NB, pl.RT);
+    int64_t ns = (d->max_smem_optin - fixed) / pl.slot_bytes;
+    if (ns > kGemvMaxSlots) ns = kGemvMaxSlots;
+    if (ns > pl.nstage) ns = pl.nstage;
+    if (ns >= 2 || (ns >= 1 && pl.nstage == 1)) {
+      p.nslots = static_cast<int>(ns);
+      const size_t smem = static_cast<size_t>(
+          gemv_dyn_smem_bytes(pl.sc_bytes, pl.slot_bytes, p.nslots, pl.nstage, pl.NB, pl.RT));
+      auto k = a.yt == TB_FP32 ? gemv_2bit_dyn_kernel<float> : gemv_2bit_dyn_kernel<__nv_bfloat16>;
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
+      return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), smem, a.st, tm, p);
+    }
+  }
   switch (static_cast<int>(a.M)) {
     case 1: return launch_gemv<1>(a, d, pl, tm, p);
     case 2: return launch_gemv<2>(a, d, pl, tm, p);
