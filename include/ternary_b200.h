@@ -34,6 +34,12 @@
  *   - Calls are thread-safe.  The only library state is a per-device cache of
  *     device attributes and one per-device fault word (see
  *     tb_get_device_fault).
+ *   - Kernels are launched with programmatic dependent launch: a call may
+ *     start reading its packed weights, scales and signs while the previous
+ *     kernel on the stream is still running (activations and outputs wait for
+ *     it).  Weights, scales and signs are layer constants; they must not be
+ *     written by a kernel that lets its dependents launch early (the library's
+ *     own pack kernel, like any plain kernel or copy, does not).
  *
  * Packed formats (codes only; the FP16 scales always live in a separate
  * [N, K/128] array, row-major, scale g of row n covering k = 128g..128g+127):
@@ -87,9 +93,10 @@ typedef int tb_dtype;
 
 typedef int tb_path;
 #define TB_PATH_AUTO 0   /* choose by shape (what tb_ternary_linear does)       */
-#define TB_PATH_GEMV 1   /* CUDA-core streaming kernel (dp4a on 16-bit fixed-point
-                            activations), for M <= 4; for M * K/1024 <= 16 the
-                            rotation runs inside it (one launch per call)       */
+#define TB_PATH_GEMV 1   /* CUDA-core streaming kernels on 16-bit fixed-point
+                            activations, for M <= 4 (base-3: M <= 16).  One token
+                            (2-bit): an L2-prefetch launch, then the decode
+                            kernel, which rotates x itself for K <= 32768      */
 #define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
                             s*t in shared memory, fp32 accumulators in TMEM)    */
 #define TB_PATH_SIMPLE 3 /* plain per-row kernel: any K % 128, any alignment    */
@@ -145,8 +152,9 @@ size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K)
 /* y = x' W^T with W the ternary g128 matrix given by (packed, scales, f).
  *   x       : device [M, K].  xt in {BF16, FP16, FP32}: float mode; xt = INT8:
  *             integer mode.
- *   signs   : device [K] int8 or NULL.  Non-NULL: x is unrotated and the
- *             rotation x' = R^T x is applied first (needs K % 1024 == 0).
+ *   signs   : device [K] int8, each -1 or +1, or NULL.  Non-NULL: x is
+ *             unrotated and the rotation x' = R^T x is applied first (needs
+ *             K % 1024 == 0).
  *             NULL: x is taken as already rotated.  Must be NULL in integer mode.
  *   scales  : device [N, K/128] fp16 bit patterns.  Ignored in integer mode.
  *   y       : device [M, N]; yt in {FP32, BF16} in float mode, INT32 in integer

@@ -97,23 +97,14 @@ __host__ __device__ inline int64_t gemv_smem_bytes(int64_t sc_bytes, int64_t slo
   return 1024 + sc_bytes + slot_bytes * nslots + 8 * (kGemvMaxSlots + 1) + 4 * kGemvMaxSlots;
 }
 
-// Activation prep: grid (K/1024, M), 128 threads per (1024-block, token);
-// thread t holds elements 8t .. 8t+7 of the block (the 128-thread block
-// transform of hadamard.cuh), so a 128-group is 16 threads and thread pair
-// (2i, 2i+1) of a group holds its 16-code word i.  Launched with programmatic
-// dependent launch: it waits for the previous kernel on the stream (which may
-// have produced x, or may still be reading this workspace) before touching
-// either.
-template <typename TIn>
-__global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restrict__ x,
-                                                              const int8_t* __restrict__ signs,
-                                                              uint8_t* __restrict__ ws, int K, int NB) {
-  __shared__ float sm[kHB];
-  pdl_launch_dependents();
-  pdl_wait();
-  const int blk = blockIdx.x, m = blockIdx.y, M = gridDim.y, t = threadIdx.x;
-  float v[8];
-  load_rotated8<TIn>(x, signs, m, blk, K, v, sm);
+// 16-bit fixed point of one 128-group whose values are spread over 16
+// consecutive lanes of a warp, 8 each (lane u = t & 15 holds codes 8u .. 8u+7
+// of the group, the layout of the 128-thread block transform).  Writes the
+// group's 256 bytes of activation words to `gw` and, from lane u = 0, its
+// {e_g, sum of q} to `*inf`.  Word (plane p, i, j) sits at byte 128 p + 16 i +
+// 4 j, and its byte b holds plane p of code 16 i + 4 b + j: lane pair
+// (2i, 2i + 1) holds word i's codes.
+__device__ __forceinline__ void gemv_quantize_group8(const float v[8], int t, uint8_t* gw, int2* inf) {
   float mx = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
@@ -144,17 +135,38 @@ __global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restr
     const uint32_t recv = __shfl_xor_sync(0xffffffffu, h ? hh : hl, 1);
     word[j] = h ? (recv | (hl << 16)) : (hh | (recv << 16));
   }
+  *reinterpret_cast<uint4*>(gw + h * 128 + wi * 16) = make_uint4(word[0], word[1], word[2], word[3]);
+  if (u == 0) {
+    int2 i2;
+    i2.x = __float_as_int(e);
+    i2.y = qs;
+    *inf = i2;
+  }
+}
+
+// Activation prep: grid (K/1024, M), 128 threads per (1024-block, token);
+// thread t holds elements 8t .. 8t+7 of the block (the 128-thread block
+// transform of hadamard.cuh), so a 128-group is 16 threads and thread pair
+// (2i, 2i+1) of a group holds its 16-code word i.  Launched with programmatic
+// dependent launch: it waits for the previous kernel on the stream (which may
+// have produced x, or may still be reading this workspace) before touching
+// either.
+template <typename TIn>
+__global__ void __launch_bounds__(kHThreads) prep_gemv_kernel(const TIn* __restrict__ x,
+                                                              const int8_t* __restrict__ signs,
+                                                              uint8_t* __restrict__ ws, int K, int NB) {
+  __shared__ float sm[kHB];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int blk = blockIdx.x, m = blockIdx.y, M = gridDim.y, t = threadIdx.x;
+  float v[8];
+  load_rotated8<TIn>(x, signs, m, blk, K, v, sm);
   const int g = blk * 8 + (t >> 4);  // global group index
   const int s = g / (4 * NB), gs = g % (4 * NB);
   uint8_t* blkbase = ws + static_cast<int64_t>(s) * gemv_act_stage_bytes(M, NB);
   uint8_t* gw = blkbase + (static_cast<int64_t>(m) * 4 * NB + gs) * kGemvGroupBytes;
-  *reinterpret_cast<uint4*>(gw + h * 128 + wi * 16) = make_uint4(word[0], word[1], word[2], word[3]);
-  if (u == 0) {
-    int2 inf;
-    inf.x = __float_as_int(e);
-    inf.y = qs;
-    reinterpret_cast<int2*>(blkbase + static_cast<int64_t>(M) * 4 * NB * kGemvGroupBytes)[m * 4 * NB + gs] = inf;
-  }
+  int2* inf = reinterpret_cast<int2*>(blkbase + static_cast<int64_t>(M) * 4 * NB * kGemvGroupBytes) + m * 4 * NB + gs;
+  gemv_quantize_group8(v, t, gw, inf);
 }
 
 // Integer group sum  sum_k c_k q_k  of one item for one token, mask mode (a

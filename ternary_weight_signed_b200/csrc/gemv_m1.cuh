@@ -1,0 +1,469 @@
+// Decode GEMV for one token (M = 1) on the 2-bit slot format, sized so that
+// two CTAs share an SM.
+//
+// y[n] = sum_g s[n, g] * sum_{k in g} t[n, k] x'[k]   (ternary g128;
+// news.ditty.ir, "Bonsai 2 27B", second paragraph; ai4coding.ru, "What is a
+// ternary model": the ternary product is an add, a subtract or nothing).
+//
+// Arithmetic.  x' is held per 128-group as 16-bit fixed point
+// q = rint(x' / e_g), e_g = max|x'_g| / 32512.  A packed word w holds 16 codes
+// (code 4b + j of the word in bits 8b + 2j); masking it with 0x03030303 << 2j
+// leaves the biased codes c = t + 1 of slot j, times 4^j, one per byte.
+// dp2a multiplies two of those bytes by two int16 values of q, so
+//   T_j = sum over the group's words of 4^j c q   (exact in int32),
+//   sum_k t q = T_0 + T_1 / 4 + T_2 / 16 + T_3 / 64 - sum_k q,
+// and the group adds s[n, g] * e_g * (that) to row n's fp32 sum.
+//
+// Activation words of a group (256 bytes, 64 words): word 8 i + 2 j + h holds
+// the int16 values of codes 16 i + 8 h + j (low half) and 16 i + 8 h + 4 + j
+// (high half): what dp2a.lo (h = 0) and dp2a.hi (h = 1) pair with bytes 0, 1
+// and 2, 3 of the slot-j mask of packed word i.  Then per group {e_g, sum q}.
+//
+// Rotation (news.ditty.ir, second and third paragraphs; openbonsai.org, "How
+// it works", "Rotate"): x'_b = H (d_b * x_b) / 32 on each 1024-block, H the
+// Sylvester matrix.  One warp rotates one block: lane a holds elements
+// 32 a .. 32 a + 31; the transform over the low five index bits runs inside
+// the lane, over the high five bits across lanes (butterflies by shuffle), so
+// lane a ends with x'[32 a .. 32 a + 31], a quarter of group a / 4.  The 1/32
+// is exact and is folded into the fixed-point scale.
+//
+// Overlap of consecutive calls.  Each call is two launches, both with
+// programmatic dependent launch: gemv1_prefetch_kernel (one 32-thread CTA per
+// decode CTA) starts as soon as the previous call's decode kernel begins,
+// asks L2 to fetch this call's packed weights and scales, and then waits for
+// the previous kernel to finish; the decode kernel (one 16-warp CTA per SM,
+// registers and shared memory capped so that the next call's prefetch CTA
+// fits beside it) follows.  HBM therefore keeps streaming the next call's
+// weights while this call computes.  Packed weights, scales and signs are read
+// before the wait for the previous kernel: they must not be written by a
+// kernel that itself lets its dependents launch early.
+//
+// With `kFused` the decode CTA rotates x itself (one warp per 1024-block): no
+// workspace.  Otherwise prep_gemv1_kernel writes the activation words to the
+// workspace and one bulk copy brings them.
+//
+// Work split.  A CTA owns R consecutive rows; a 512-code chunk is 128 bytes of
+// each (one TMA box, 128-byte swizzle); stages of NB chunks go through a ring
+// of slots (usually all of them at once).  Rows come in tiles of 8: lane l
+// works on row 8 t + (l & 7) of a tile and group slot l >> 3 of a chunk, so
+// each quarter-warp holds one group's activation words (broadcast loads) and
+// its eight lanes read eight rows whose swizzled 16-byte pieces fall in eight
+// different bank groups.  Warp w < Wt * Wk owns row-tile group w / Wk (at most
+// TPW tiles) and the chunks c = w % Wk (mod Wk), keeps one fp32 sum per tile
+// in registers over all of its chunks, and runs two tiles at a time.  At the
+// end the four group slots of a row are added by shuffles and the Wk warps of
+// a tile group in order of w: the result does not depend on timing (bitwise
+// reproducible).
+#pragma once
+#include "gemv.cuh"
+#include "hadamard.cuh"
+#include "tb_device.cuh"
+
+namespace tb {
+
+constexpr int kG1Warps = 16;
+constexpr int kG1Threads = 32 * kG1Warps;
+constexpr int kG1MaxRegs = 120;  // 16 warps x 120 leaves registers for a prefetch CTA
+// Dynamic shared memory of a decode CTA at most (the SM's 228 KB less room for
+// a prefetch CTA and the per-CTA reservations).
+constexpr int kG1SmemMax = 220 * 1024;
+constexpr int kG1MaxRows = 256;  // TMA box height limit
+// The CTA rotates x itself for K up to this many 1024-blocks (two per warp).
+constexpr int kG1FusedMaxBlocks = 2 * kG1Warps;
+constexpr int kG1GroupBytes = 256;
+constexpr int kG1PrefetchPiece = 64 * 1024;
+
+// d = c + a.lo16 * b.byte0 + a.hi16 * b.byte1 (lo) or * bytes 2, 3 (hi);
+// a signed 16-bit, b unsigned 8-bit.
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// L2 prefetch of `bytes` at `p` (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+struct Gemv1Params {
+  const void* x;           // [K] activations (fused) or nullptr
+  const int8_t* signs;     // [K] or nullptr (x already rotated)
+  const uint8_t* act;      // prep_gemv1_kernel output (not fused)
+  const uint16_t* scales;  // [N, K/128] fp16 bits
+  void* y;                 // [N]
+  int N, K;
+  int R;                   // rows per CTA (TMA box height)
+  int RT;                  // row tiles of 8 covering R
+  int Wt, Wk;              // row-tile groups x chunk classes <= kG1Warps
+  int NB;                  // chunks (boxes) per stage
+  int nstage, nslots;
+  int box_stride;          // bytes between boxes (R * 128 rounded up to 1 KB)
+  int slot_bytes;          // NB * box_stride
+  int off_act, off_sc, off_red, off_bar;  // shared-memory offsets from the 1 KB-aligned base
+};
+
+// Shared memory (offsets from the 1 KB-aligned base; 1 KB of slack in front):
+//   ring  nslots x slot_bytes
+//   act   G x 256 bytes of activation words, then G x {float e_g, int sum q}
+//   sc    R x G fp16 scales of the CTA's rows
+//   red   Wk x R fp32 row sums of the warps
+//   bar   full[nstage], pre_bar; counters done[nstage], issued[nstage], fault
+struct Gemv1Layout {
+  int off_act, off_sc, off_red, off_bar;
+  int64_t bytes;
+};
+__host__ __device__ inline int64_t g1_act_bytes(int64_t K) { return (K / 128) * (kG1GroupBytes + 8); }
+__host__ __device__ inline Gemv1Layout gemv1_layout(int64_t K, int R, int Wk, int nstage, int64_t ring_bytes) {
+  const int64_t G = K / 128;
+  Gemv1Layout l;
+  l.off_act = static_cast<int>(ring_bytes);
+  l.off_sc = static_cast<int>(l.off_act + align128(g1_act_bytes(K)));
+  l.off_red = static_cast<int>(l.off_sc + align128(static_cast<int64_t>(R) * G * 2));
+  l.off_bar = static_cast<int>(l.off_red + align128(static_cast<int64_t>(Wk) * R * 4));
+  l.bytes = 1024 + l.off_bar + 8 * (nstage + 1) + 4 * (2 * nstage + 1);
+  return l;
+}
+
+// ---------------------------------------------------------------- rotation
+// The lane's 32 signs of block `blk` as packed bytes (loaded before the wait
+// for the previous kernel: signs are parameters of the layer).
+__device__ __forceinline__ void g1_load_signs(const int8_t* signs, int blk, int lane, uint32_t (&sg)[8]) {
+  const uint4* p = reinterpret_cast<const uint4*>(signs + static_cast<int64_t>(blk) * kHB + 32 * lane);
+  const uint4 a = p[0], b = p[1];
+  sg[0] = a.x; sg[1] = a.y; sg[2] = a.z; sg[3] = a.w;
+  sg[4] = b.x; sg[5] = b.y; sg[6] = b.z; sg[7] = b.w;
+}
+
+template <typename T>
+__device__ __forceinline__ void g1_load32(const T* p, float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) load8<T>(p + 8 * i, v + 8 * i);
+}
+
+// One warp: rotate 1024-block `blk` (with signs `sg` when has_signs, else
+// x is taken as already rotated) and write its 8 groups' activation words and
+// info into `act` (G groups of words, then G infos).
+template <typename TIn>
+__device__ __forceinline__ void g1_rotate_block(const TIn* __restrict__ x, const uint32_t (&sg)[8], bool has_signs,
+                                                int blk, int G, uint8_t* act, int lane) {
+  float v[32];
+  g1_load32<TIn>(x + static_cast<int64_t>(blk) * kHB + 32 * lane, v);
+  float scale = 1.f;
+  if (has_signs) {
+    // sign byte 0xFF (-1) flips the float's sign bit
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t sbit = (sg[i >> 2] << (24 - 8 * (i & 3))) & 0x80000000u;
+      v[i] = __int_as_float(__float_as_int(v[i]) ^ static_cast<int>(sbit));
+    }
+    // low five index bits: inside the lane
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if ((i & h) == 0) {
+          const float a = v[i], b = v[i + h];
+          v[i] = a + b;
+          v[i + h] = a - b;
+        }
+      }
+    }
+    // high five index bits: across lanes (lower partner keeps a + b, upper gets a - b)
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const float sgn = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn, v[i], __shfl_xor_sync(0xffffffffu, v[i], m));
+    }
+    scale = kHNorm;
+  }
+  // 16-bit fixed point of the group (4 lanes): e = max|x'| / kQMax with x' = scale * v
+  float mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(v[i]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  mx *= scale;  // exact (a power of two)
+  const float e = mx / kQMax;
+  // inv * scale is exact too, so q = rint(x' * kQMax / max|x'|) as in prep_gemv_kernel
+  const float inv = mx > 0.f ? (kQMax / mx) * scale : 0.f;
+  int q[32];
+  int qs = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    q[i] = max(-32512, min(32512, __float2int_rn(v[i] * inv)));
+    qs += q[i];
+  }
+  qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+  qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+  // lane a holds codes 32 (a & 3) .. + 31 of group a >> 2, i.e. words
+  // i = 2 (a & 3) + i2 (i2 = 0, 1); word 8 i + 2 j + h pairs codes
+  // 16 i + 8 h + j and 16 i + 8 h + 4 + j
+  uint32_t wv[16];
+#pragma unroll
+  for (int i2 = 0; i2 < 2; ++i2)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int u = 16 * i2 + 8 * h + j;
+        wv[8 * i2 + 2 * j + h] = __byte_perm(static_cast<uint32_t>(q[u]), static_cast<uint32_t>(q[u + 4]), 0x5410);
+      }
+  const int g = blk * 8 + (lane >> 2);
+  uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupBytes + 64 * (lane & 3));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+  if ((lane & 3) == 0) {
+    int2 inf;
+    inf.x = __float_as_int(e);
+    inf.y = qs;
+    reinterpret_cast<int2*>(act + G * kG1GroupBytes)[g] = inf;
+  }
+}
+
+// Activation words for long K: one warp per 1024-block, 4 warps per CTA,
+// written to `ws` in the layout above.  Waits for the previous kernel on the
+// stream (which may have produced x, or may still read ws) before touching
+// either.
+template <typename TIn>
+__global__ void __launch_bounds__(128) prep_gemv1_kernel(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
+                                                         uint8_t* __restrict__ ws, int K) {
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int blk = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const bool live = blk < (K >> 10);
+  uint32_t sg[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (live && signs != nullptr) g1_load_signs(signs, blk, lane, sg);
+  pdl_wait();
+  if (live) g1_rotate_block<TIn>(x, sg, signs != nullptr, blk, K >> 7, ws, lane);
+}
+
+// ---------------------------------------------------------------- prefetch
+// One 32-thread CTA per decode CTA: L2 prefetch of the decode CTA's packed
+// rows and scales (contiguous in memory), then a wait for the previous kernel
+// on the stream, so that the decode kernel's own wait (for this kernel) also
+// covers that one.
+__global__ void __launch_bounds__(32) gemv1_prefetch_kernel(const uint8_t* __restrict__ packed,
+                                                            const uint16_t* __restrict__ scales, int N, int K, int R) {
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    const int r0 = blockIdx.x * R;
+    const int rows = min(R, N - r0);
+    const int64_t row_bytes = K / 4;
+    const uint8_t* w = packed + static_cast<int64_t>(r0) * row_bytes;
+    const int64_t wbytes = static_cast<int64_t>(rows) * row_bytes;
+    for (int64_t o = 0; o < wbytes; o += kG1PrefetchPiece)
+      prefetch_l2(w + o, static_cast<uint32_t>(wbytes - o < kG1PrefetchPiece ? wbytes - o : kG1PrefetchPiece));
+    prefetch_l2(scales + static_cast<int64_t>(r0) * (K / 128), static_cast<uint32_t>(rows * (K / 128) * 2));
+  }
+  pdl_wait();
+}
+
+// ---------------------------------------------------------------- decode
+// Stage s: its chunks' weight boxes into slot `slot`, completing on `bar`.
+__device__ __forceinline__ void gemv1_issue(const CUtensorMap* tm, const Gemv1Params& p, uint8_t* ring,
+                                            uint64_t* bar, int s, int slot, int r0) {
+  const int C = p.K >> 9;
+  const int nb = min(p.NB, C - s * p.NB);
+  uint8_t* dst = ring + static_cast<int64_t>(slot) * p.slot_bytes;
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb) * static_cast<uint32_t>(p.R) * 128u);
+  for (int b = 0; b < nb; ++b) tma_load_2d(dst + b * p.box_stride, tm, (s * p.NB + b) * 128, r0, bar);
+}
+
+// sum_k c_k q_k of one row's group: 8 packed words against the group's 64
+// activation words (the four T_j combined exactly).
+__device__ __forceinline__ int g1_group_dot(const uint4& wa, const uint4& wb, const uint32_t (&A)[64]) {
+  const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+  int lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t c = w[i] & (0x03030303u << (2 * j));
+      lo[j] = dp2a_lo(A[8 * i + 2 * j], c, lo[j]);
+      hi[j] = dp2a_hi(A[8 * i + 2 * j + 1], c, hi[j]);
+    }
+  }
+  return (lo[0] + hi[0]) + ((lo[1] + hi[1]) >> 2) + ((lo[2] + hi[2]) >> 4) + ((lo[3] + hi[3]) >> 6);
+}
+
+// TPW: row tiles per warp at most (1, 2 or 4).
+template <typename TIn, typename TOut, bool kFused, int TPW>
+__global__ void __maxnreg__(kG1MaxRegs)
+    gemv1_2bit_kernel(const __grid_constant__ CUtensorMap tm_w, const Gemv1Params p) {
+  pdl_launch_dependents();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* ring = base;
+  uint8_t* act = base + p.off_act;
+  const __half* sc = reinterpret_cast<const __half*>(base + p.off_sc);
+  float* red = reinterpret_cast<float*>(base + p.off_red);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + p.off_bar);
+  uint64_t* pre_bar = full + p.nstage;  // scales (+ activation words when not fused)
+  uint32_t* done = reinterpret_cast<uint32_t*>(pre_bar + 1);  // warps finished with stage s
+  uint32_t* issued = done + p.nstage;                          // 1 once stage s was issued
+  uint32_t* cta_fault = issued + p.nstage;
+
+  const int G = p.K >> 7, C = p.K >> 9;
+  const int r0 = blockIdx.x * p.R;
+  const int nrows = min(p.R, p.N - r0);
+  const int pre = min(p.nslots, p.nstage);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tm_w);
+    for (int s = 0; s < p.nstage; ++s) {
+      mbar_init(&full[s], 1);
+      done[s] = 0;
+      issued[s] = s < pre ? 1u : 0u;
+    }
+    *cta_fault = 0;
+    mbar_init(pre_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // The weights do not depend on earlier work on the stream.  Issuing a TMA
+  // copy takes a while, so the stages are spread over the warps' lane 0 (the
+  // last warps first: the first warps rotate x).
+  if (lane == 0) {
+    if (warp == kG1Warps - 1) {
+      const uint32_t sbytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(G * 2);
+      const uint32_t abytes = kFused ? 0u : static_cast<uint32_t>(g1_act_bytes(p.K));
+      mbar_arrive_expect_tx(pre_bar, sbytes + abytes);
+      bulk_load(base + p.off_sc, p.scales + static_cast<int64_t>(r0) * G, sbytes, pre_bar);
+    }
+    for (int s = kG1Warps - 1 - warp; s < pre; s += kG1Warps) gemv1_issue(&tm_w, p, ring, &full[s], s, s, r0);
+    if constexpr (!kFused) {
+      if (warp == kG1Warps - 1) {
+        pdl_wait();  // the prep kernel's activation words
+        bulk_load(act, p.act, static_cast<uint32_t>(g1_act_bytes(p.K)), pre_bar);
+      }
+    }
+  }
+  if constexpr (kFused) {
+    const int nblk = p.K >> 10;
+    uint32_t sg0[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sg1[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const bool b0 = warp < nblk, b1 = warp + kG1Warps < nblk;
+    if (p.signs != nullptr) {
+      if (b0) g1_load_signs(p.signs, warp, lane, sg0);
+      if (b1) g1_load_signs(p.signs, warp + kG1Warps, lane, sg1);
+    }
+    pdl_wait();  // x may be the previous kernel's output
+    const TIn* x = static_cast<const TIn*>(p.x);
+    if (b0) g1_rotate_block<TIn>(x, sg0, p.signs != nullptr, warp, G, act, lane);
+    if (b1) g1_rotate_block<TIn>(x, sg1, p.signs != nullptr, warp + kG1Warps, G, act, lane);
+  }
+  __syncthreads();
+
+  const int rsub = lane & 7, gslot = lane >> 3;
+  const int tg = warp / p.Wk, wk = warp - tg * p.Wk;
+  const bool active = tg < p.Wt;
+  const int t0 = tg * p.RT / p.Wt, nt = active ? (tg + 1) * p.RT / p.Wt - t0 : 0;  // this warp's row tiles
+  const int2* info = reinterpret_cast<const int2*>(act + G * kG1GroupBytes);
+  // byte offsets of the lane's rows in a box (the group's two 16-byte pieces
+  // 2 gslot, 2 gslot + 1, swizzled with the row index mod 8 = rsub) and of
+  // the rows' scales; rows past the CTA's end read valid rows, sums dropped
+  const int u0 = ((2 * gslot) ^ rsub) << 4, u1 = ((2 * gslot + 1) ^ rsub) << 4;
+  int roff[TPW], soff[TPW];
+  float acc[TPW];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    const int r = 8 * (t0 + i) + rsub;
+    roff[i] = min(r, p.R - 1) * 128;
+    soff[i] = min(r, nrows - 1) * G;
+    acc[i] = 0.f;
+  }
+
+  bool ok = __all_sync(0xffffffffu, mbar_wait_backoff(pre_bar, 0, FAULT_WAIT_ACT));
+  int c = active ? wk : C;  // this warp's next chunk
+  for (int s = 0; s < p.nstage && ok; ++s) {
+    const int cend = min(C, (s + 1) * p.NB);
+    if (c < cend) {
+      ok = __all_sync(0xffffffffu, mbar_wait_backoff(&full[s], 0, FAULT_WAIT_FULL)) &&
+           *reinterpret_cast<volatile uint32_t*>(cta_fault) == 0u;
+      if (!ok) break;
+      const uint8_t* slot = ring + static_cast<int64_t>(s % p.nslots) * p.slot_bytes;
+      const int cbeg = s * p.NB;
+      for (; c < cend; c += p.Wk) {
+        const int g = 4 * c + gslot;
+        uint32_t A[64];
+        const uint4* src = reinterpret_cast<const uint4*>(act + g * kG1GroupBytes);
+#pragma unroll
+        for (int v = 0; v < 16; ++v) {
+          const uint4 u4 = src[v];
+          A[4 * v] = u4.x;
+          A[4 * v + 1] = u4.y;
+          A[4 * v + 2] = u4.z;
+          A[4 * v + 3] = u4.w;
+        }
+        const int2 inf = info[g];
+        const float e = __int_as_float(inf.x);
+        const uint8_t* box = slot + (c - cbeg) * p.box_stride;
+        if constexpr (TPW == 1) {
+          const uint4 w0 = *reinterpret_cast<const uint4*>(box + roff[0] + u0);
+          const uint4 w1 = *reinterpret_cast<const uint4*>(box + roff[0] + u1);
+          const float sa = __half2float(sc[soff[0] + g]) * e;
+          acc[0] = fmaf(__int2float_rn(g1_group_dot(w0, w1, A) - inf.y), sa, acc[0]);
+        } else {
+#pragma unroll
+          for (int tp = 0; tp < TPW; tp += 2) {
+            // tiles beyond nt compute on valid rows and are dropped at the end
+            const uint4 wa0 = *reinterpret_cast<const uint4*>(box + roff[tp] + u0);
+            const uint4 wa1 = *reinterpret_cast<const uint4*>(box + roff[tp] + u1);
+            const uint4 wb0 = *reinterpret_cast<const uint4*>(box + roff[tp + 1] + u0);
+            const uint4 wb1 = *reinterpret_cast<const uint4*>(box + roff[tp + 1] + u1);
+            const float sa = __half2float(sc[soff[tp] + g]) * e;
+            const float sb = __half2float(sc[soff[tp + 1] + g]) * e;
+            const int da = g1_group_dot(wa0, wa1, A) - inf.y;
+            const int db = g1_group_dot(wb0, wb1, A) - inf.y;
+            acc[tp] = fmaf(__int2float_rn(da), sa, acc[tp]);
+            acc[tp + 1] = fmaf(__int2float_rn(db), sb, acc[tp + 1]);
+          }
+        }
+      }
+    }
+    // the warp completing stage s refills its slot with stage s + nslots
+    if (p.nslots < p.nstage) {
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        if (atomicAdd(&done[s], 1u) == static_cast<uint32_t>(kG1Warps - 1) && s + p.nslots < p.nstage) {
+          __threadfence_block();
+          issued[s + p.nslots] = 1u;
+          gemv1_issue(&tm_w, p, ring, &full[s + p.nslots], s + p.nslots, s % p.nslots, r0);
+        }
+      }
+    }
+  }
+  if (!ok && lane == 0) atomicExch(cta_fault, 1u);  // the other warps stop at their next stage
+  // row sums of this warp: the chunk's four group slots (lanes rsub + 8 k)
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    float v = acc[i];
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    const int r = 8 * (t0 + i) + rsub;
+    if (i < nt && gslot == 0 && r < p.R) red[wk * p.R + r] = v;
+  }
+  __syncthreads();
+  // After a wait that gave up, copies may still be in flight into the ring:
+  // wait (bounded) for every issued stage before the CTA exits.
+  if (threadIdx.x == 0 && *cta_fault != 0) {
+    for (int s = 0; s < p.nstage; ++s)
+      if (issued[s] && !mbar_wait(&full[s], 0, FAULT_WAIT_FULL)) break;
+  }
+  TOut* y = reinterpret_cast<TOut*>(p.y);
+  for (int r = threadIdx.x; r < nrows; r += kG1Threads) {
+    float sum = 0.f;
+    for (int k = 0; k < p.Wk; ++k) sum += red[k * p.R + r];
+    y[r0 + r] = from_f32<TOut>(sum);
+  }
+}
+
+}  // namespace tb

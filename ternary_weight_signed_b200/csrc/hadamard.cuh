@@ -152,22 +152,32 @@ __device__ __forceinline__ void fwht1024(float v[8], float* sm) { fwht1024_group
 
 // Loads the thread's 8 elements of block `blk` of row `row`, applies the
 // forward rotation (signs, transform, 1/32) when `signs` is non-null, else
-// only converts to fp32.  All 128 threads must call.
+// only converts to fp32.  Called by all 128 threads of a group: `t` is the
+// thread's index in the group, `bar` the group's named barrier (see
+// fwht1024_group).
 template <typename TIn>
-__device__ __forceinline__ void load_rotated8(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
-                                              int64_t row, int blk, int64_t K, float v[8],
-                                              float* sm) {
-  const int64_t k0 = static_cast<int64_t>(blk) * kHB + 8 * threadIdx.x;
+__device__ __forceinline__ void load_rotated8_group(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
+                                                    int64_t row, int blk, int64_t K, float v[8], float* sm,
+                                                    int t, int bar) {
+  const int64_t k0 = static_cast<int64_t>(blk) * kHB + 8 * t;
   load8_any<TIn>(x + row * K + k0, v);
   if (signs != nullptr) {
     float d[8];
     load_signs8(signs + k0, d);
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] *= d[i];
-    fwht1024(v, sm);
+    fwht1024_group(v, sm, t, bar);
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] *= kHNorm;
   }
+}
+
+// load_rotated8_group over a whole 128-thread block.
+template <typename TIn>
+__device__ __forceinline__ void load_rotated8(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
+                                              int64_t row, int blk, int64_t K, float v[8],
+                                              float* sm) {
+  load_rotated8_group<TIn>(x, signs, row, blk, K, v, sm, threadIdx.x, 0);
 }
 
 // ---------------------------------------------------------------------------

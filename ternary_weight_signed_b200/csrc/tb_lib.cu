@@ -15,6 +15,7 @@
 
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_m1.cuh"
 #include "gemv_b3.cuh"
 #include "gemv_tc.cuh"
 #include "hadamard.cuh"
@@ -276,6 +277,65 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, Gemv
   return true;
 }
 
+struct G1Plan {
+  int grid, R, RT, Wt, Wk, TPW, NB, nstage, nslots, box_stride, slot_bytes;
+  bool fused;
+  Gemv1Layout lay;
+};
+
+// Geometry of the one-token decode kernel (gemv_m1.cuh); false if it does not fit.
+bool g1_plan(int64_t N, int64_t K, int sm_count, int max_smem, bool fused, G1Plan* out) {
+  if (K % 1024 != 0 || K < 1024 || N < 1 || sm_count < 1) return false;
+  if (fused && K / kHB > kG1FusedMaxBlocks) return false;
+  G1Plan pl;
+  int64_t R = (N + sm_count - 1) / sm_count;
+  if (R > kG1MaxRows) R = kG1MaxRows;
+  pl.R = static_cast<int>(R);
+  pl.RT = static_cast<int>((R + 7) / 8);
+  pl.grid = static_cast<int>((N + R - 1) / R);
+  const int64_t C = K / 512;
+  // Wt row-tile groups x Wk chunk classes (<= kG1Warps warps): the least
+  // issue work for the busiest warp; a warp's tiles run two at a time and its
+  // activation words are loaded once per chunk
+  int64_t best_cost = -1;
+  for (int wt = 1; wt <= kG1Warps; ++wt) {
+    for (int wk = 1; wt * wk <= kG1Warps; ++wk) {
+      const int64_t tpw = (pl.RT + wt - 1) / wt;
+      if (tpw > 4) continue;
+      const int tpl = tpw == 1 ? 1 : (tpw == 2 ? 2 : 4);  // kernel instance
+      const int64_t cost = ((C + wk - 1) / wk) * (tpl * 110 + 20);
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        pl.Wt = wt;
+        pl.Wk = wk;
+        pl.TPW = tpl;
+      }
+    }
+  }
+  if (best_cost < 0) return false;
+  pl.box_stride = static_cast<int>(align_up(R * 128, 1024));
+  // stages of at least 8 KB of weights
+  int64_t nb = (8192 + R * 128 - 1) / (R * 128);
+  if (nb > C) nb = C;
+  if (nb < 1) nb = 1;
+  pl.NB = static_cast<int>(nb);
+  pl.nstage = static_cast<int>((C + nb - 1) / nb);
+  pl.slot_bytes = static_cast<int>(nb) * pl.box_stride;
+  pl.fused = fused;
+  const int64_t budget = std::min<int64_t>(kG1SmemMax, max_smem);
+  const Gemv1Layout l0 = gemv1_layout(K, pl.R, pl.Wk, pl.nstage, 0);
+  int64_t ns = (budget - l0.bytes) / pl.slot_bytes;
+  if (ns > pl.nstage) ns = pl.nstage;
+  if (ns < 1 || ns < std::min<int64_t>(2, pl.nstage)) return false;
+  pl.nslots = static_cast<int>(ns);
+  pl.lay = gemv1_layout(K, pl.R, pl.Wk, pl.nstage, ns * pl.slot_bytes);
+  if (pl.lay.bytes > budget) return false;
+  *out = pl;
+  return true;
+}
+
+bool g1_fused(int64_t K) { return K / kHB <= kG1FusedMaxBlocks; }
+
 struct B3Plan {
   int grid, R, RT, NB, nstage, nslots, box_stride, slot_bytes, sc_bytes;
   size_t smem;
@@ -385,6 +445,10 @@ bool gemv_ok(const LinearArgs& a) {
     B3Plan pl;
     return b3_plan(std::min<int64_t>(a.M, kGemvMaxM), a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
   }
+  if (a.M == 1) {
+    G1Plan p1;
+    if (g1_plan(a.N, a.K, kB200Sms, kB200SmemOptin, g1_fused(a.K), &p1)) return true;
+  }
   GemvPlan pl;
   return gemv_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
 }
@@ -427,8 +491,72 @@ tb_status launch_gemv(const LinearArgs& a, const DevInfo* d, const GemvPlan& pl,
   return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, tm, p);
 }
 
+// One token: gemv1_prefetch_kernel, then gemv1_2bit_kernel, with the rotation
+// inside the decode kernel for K up to kG1FusedMaxBlocks 1024-blocks, else
+// prep_gemv1_kernel before it.
+template <typename TIn, typename TOut, bool kFused>
+tb_status launch_gemv1(const LinearArgs& a, const DevInfo* d, const G1Plan& pl, const CUtensorMap& tm,
+                       const Gemv1Params& p) {
+  auto pick = [&]() {
+    switch (pl.TPW) {
+      case 1: return gemv1_2bit_kernel<TIn, TOut, kFused, 1>;
+      case 2: return gemv1_2bit_kernel<TIn, TOut, kFused, 2>;
+      default: return gemv1_2bit_kernel<TIn, TOut, kFused, 4>;
+    }
+  };
+  auto k = pick();
+  if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
+  return launch_pdl(k, dim3(pl.grid), dim3(kG1Threads), static_cast<size_t>(pl.lay.bytes), a.st, tm, p);
+}
+
+template <typename TIn>
+tb_status run_gemv1_typed(const LinearArgs& a, const DevInfo* d, const G1Plan& pl) {
+  CUtensorMap tm;
+  if (make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.packed, a.K / 4, a.N, a.K / 4, 128,
+                  static_cast<uint32_t>(pl.R), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+    return TB_ERR_CUDA;
+  Gemv1Params p;
+  p.x = pl.fused ? a.x : nullptr;
+  p.signs = a.signs;
+  p.act = static_cast<const uint8_t*>(a.ws);
+  p.scales = a.scales;
+  p.y = a.y;
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.R = pl.R;
+  p.RT = pl.RT;
+  p.Wt = pl.Wt;
+  p.Wk = pl.Wk;
+  p.NB = pl.NB;
+  p.nstage = pl.nstage;
+  p.nslots = pl.nslots;
+  p.box_stride = pl.box_stride;
+  p.slot_bytes = pl.slot_bytes;
+  p.off_act = pl.lay.off_act;
+  p.off_sc = pl.lay.off_sc;
+  p.off_red = pl.lay.off_red;
+  p.off_bar = pl.lay.off_bar;
+  if (launch_pdl(gemv1_prefetch_kernel, dim3(pl.grid), dim3(32), 0, a.st, a.packed, a.scales, p.N, p.K, p.R) !=
+      TB_OK)
+    return TB_ERR_CUDA;
+  if (!pl.fused) {
+    const dim3 pgrid(static_cast<unsigned>((a.K / kHB + 3) / 4));
+    if (launch_pdl(prep_gemv1_kernel<TIn>, pgrid, dim3(128), 0, a.st, static_cast<const TIn*>(a.x), a.signs,
+                   static_cast<uint8_t*>(a.ws), static_cast<int>(a.K)) != TB_OK)
+      return TB_ERR_CUDA;
+    return a.yt == TB_FP32 ? launch_gemv1<TIn, float, false>(a, d, pl, tm, p)
+                           : launch_gemv1<TIn, __nv_bfloat16, false>(a, d, pl, tm, p);
+  }
+  return a.yt == TB_FP32 ? launch_gemv1<TIn, float, true>(a, d, pl, tm, p)
+                         : launch_gemv1<TIn, __nv_bfloat16, true>(a, d, pl, tm, p);
+}
+
 template <typename TIn>
 tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
+  if (a.M == 1) {
+    G1Plan p1;
+    if (g1_plan(a.N, a.K, d->sm_count, d->max_smem_optin, g1_fused(a.K), &p1)) return run_gemv1_typed<TIn>(a, d, p1);
+  }
   GemvPlan pl;
   if (!gemv_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
   uint8_t* act = static_cast<uint8_t*>(a.ws);
