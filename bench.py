@@ -112,7 +112,7 @@ class ClockSampler:
 
 def _kernel_src_sha():
     h = hashlib.sha256()
-    for name in ("gemv.cuh", "hadamard.cuh", "tb_device.cuh"):
+    for name in ("gemv_m1.cuh", "gemv.cuh", "hadamard.cuh", "tb_device.cuh"):
         with open(os.path.join(ROOT, "ternary_weight_signed_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -135,8 +135,14 @@ def _traffic(fmt):
 
 # ---------------------------------------------------------------------------- ours
 def _launches_per_call(tb, fmt, m, n, k):
-    """Kernels one tb_ternary_linear call launches on the path it takes (all
-    float paths run an activation prep kernel and one main kernel)."""
+    """Kernels one tb_ternary_linear call launches on the path it takes: the
+    one-token 2-bit decode kernel rotates x itself up to K = 24576 (one launch);
+    the other float paths run an activation prep kernel and one main kernel."""
+    path = tb.tb_ternary_linear_path(tb.TB_BF16, fmt, m, n, k, True, True)
+    if path == tb.TB_PATH_GEMV and fmt == "2bit" and m == 1 and k // 1024 <= 24:
+        return 1
+    if path == tb.TB_PATH_GEMV and fmt == "base3":
+        return 2 * ((m + 3) // 4)
     return 2
 
 
@@ -347,7 +353,7 @@ def run_ours(args, rank, world):
     head = _decode_entry(main, peak, peak_kind, world)
     roof = head["roofline"]
     roof["traffic"] = _traffic(args.fmt)
-    roof["kernel"] = ("tb_ternary_linear decode call (prep_gemv_kernel + gemv_2bit_kernel)" if args.fmt == "2bit"
+    roof["kernel"] = ("tb_ternary_linear decode call (gemv1_2bit_kernel, rotation fused)" if args.fmt == "2bit"
                       else "tb_ternary_linear decode call (prep_b3_kernel + gemv_b3_kernel)")
     roof["timing"] = "device time per call of back-to-back calls in CUDA graphs (CUDA events on the launching stream)"
     return {

@@ -27,18 +27,17 @@
 // lane a ends with x'[32 a .. 32 a + 31], a quarter of group a / 4.  The 1/32
 // is exact and is folded into the fixed-point scale.
 //
-// Overlap of consecutive calls.  Each call is two launches, both with
-// programmatic dependent launch: gemv1_prefetch_kernel (one 32-thread CTA per
-// decode CTA) starts as soon as the previous call's decode kernel begins,
-// asks L2 to fetch this call's packed weights and scales, and then waits for
-// the previous kernel to finish; the decode kernel (one 16-warp CTA per SM,
-// registers and shared memory capped so that the next call's prefetch CTA
-// fits beside it) follows.  HBM therefore keeps streaming the next call's
-// weights while this call computes.  Packed weights, scales and signs are read
-// before the wait for the previous kernel: they must not be written by a
-// kernel that itself lets its dependents launch early.
+// Overlap of consecutive calls.  A CTA has 8 warps, at most 128 registers a
+// thread and at most 113 KB of shared memory, so the next call's CTA fits on
+// the SM beside it.  Every CTA lets its dependents launch at once
+// (programmatic dependent launch): the next call's CTA fills its own ring
+// with weights while this one computes, and only its activation work waits
+// (griddepcontrol.wait) for this call to end.  HBM therefore keeps streaming
+// across call boundaries, and a call waits on exactly one kernel boundary.
+// Packed weights, scales and signs are read before that wait: they must not
+// be written by a kernel that itself lets its dependents launch early.
 //
-// With `kFused` the decode CTA rotates x itself (one warp per 1024-block): no
+// With `kFused` the CTA rotates x itself (one or two warps per 1024-block): no
 // workspace.  Otherwise prep_gemv1_kernel writes the activation words to the
 // workspace and one bulk copy brings them.
 //
@@ -61,17 +60,14 @@
 
 namespace tb {
 
-constexpr int kG1Warps = 16;
+constexpr int kG1Warps = 8;
 constexpr int kG1Threads = 32 * kG1Warps;
-constexpr int kG1MaxRegs = 120;  // 16 warps x 120 leaves registers for a prefetch CTA
-// Dynamic shared memory of a decode CTA at most (the SM's 228 KB less room for
-// a prefetch CTA and the per-CTA reservations).
-constexpr int kG1SmemMax = 220 * 1024;
+// Shared memory per CTA for two CTAs per SM (228 KB per SM, 1 KB reserved per CTA).
+constexpr int kG1SmemMax = 115 * 1024 - 2048;
 constexpr int kG1MaxRows = 256;  // TMA box height limit
-// The CTA rotates x itself for K up to this many 1024-blocks (two per warp).
-constexpr int kG1FusedMaxBlocks = 2 * kG1Warps;
+// The CTA rotates x itself for K up to this many 1024-blocks (three per warp).
+constexpr int kG1FusedMaxBlocks = 3 * kG1Warps;
 constexpr int kG1GroupBytes = 256;
-constexpr int kG1PrefetchPiece = 64 * 1024;
 
 // d = c + a.lo16 * b.byte0 + a.hi16 * b.byte1 (lo) or * bytes 2, 3 (hi);
 // a signed 16-bit, b unsigned 8-bit.
@@ -86,11 +82,6 @@ __device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
   return d;
 }
 
-// L2 prefetch of `bytes` at `p` (16-byte aligned, multiple of 16).
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 struct Gemv1Params {
   const void* x;           // [K] activations (fused) or nullptr
   const int8_t* signs;     // [K] or nullptr (x already rotated)
@@ -101,7 +92,7 @@ struct Gemv1Params {
   int R;                   // rows per CTA (TMA box height)
   int RT;                  // row tiles of 8 covering R
   int Wt, Wk;              // row-tile groups x chunk classes <= kG1Warps
-  int NB;                  // chunks (boxes) per stage
+  int NB, nb_log2;         // chunks (boxes) per stage, a power of two
   int nstage, nslots;
   int box_stride;          // bytes between boxes (R * 128 rounded up to 1 KB)
   int slot_bytes;          // NB * box_stride
@@ -112,20 +103,25 @@ struct Gemv1Params {
 //   ring  nslots x slot_bytes
 //   act   G x 256 bytes of activation words, then G x {float e_g, int sum q}
 //   sc    R x G fp16 scales of the CTA's rows
-//   red   Wk x R fp32 row sums of the warps
+//   red   Wk x R fp32 row sums of the warps (before that, the exchange
+//         buffer of the two-warp rotation: 4 KB per 1024-block)
 //   bar   full[nstage], pre_bar; counters done[nstage], issued[nstage], fault
 struct Gemv1Layout {
   int off_act, off_sc, off_red, off_bar;
   int64_t bytes;
 };
 __host__ __device__ inline int64_t g1_act_bytes(int64_t K) { return (K / 128) * (kG1GroupBytes + 8); }
+// Two warps rotate each 1024-block when there are warps enough for that.
+__host__ __device__ constexpr bool g1_half_blocks(int64_t K) { return 2 * (K / 1024) <= kG1Warps; }
 __host__ __device__ inline Gemv1Layout gemv1_layout(int64_t K, int R, int Wk, int nstage, int64_t ring_bytes) {
   const int64_t G = K / 128;
   Gemv1Layout l;
   l.off_act = static_cast<int>(ring_bytes);
   l.off_sc = static_cast<int>(l.off_act + align128(g1_act_bytes(K)));
   l.off_red = static_cast<int>(l.off_sc + align128(static_cast<int64_t>(R) * G * 2));
-  l.off_bar = static_cast<int>(l.off_red + align128(static_cast<int64_t>(Wk) * R * 4));
+  int64_t red = static_cast<int64_t>(Wk) * R * 4;
+  if (g1_half_blocks(K) && red < (K / 1024) * 4096) red = (K / 1024) * 4096;
+  l.off_bar = static_cast<int>(l.off_red + align128(red));
   l.bytes = 1024 + l.off_bar + 8 * (nstage + 1) + 4 * (2 * nstage + 1);
   return l;
 }
@@ -227,6 +223,96 @@ __device__ __forceinline__ void g1_rotate_block(const TIn* __restrict__ x, const
   }
 }
 
+// Two warps, halves hf = 0, 1 of 1024-block `blk`: lane l of half hf holds
+// elements 512 hf + 16 l .. + 15.  Index bits 0-3 are transformed inside the
+// lane, bits 4-8 across lanes, bit 9 across the two warps through `xch` (1024
+// floats of the pair's own; named barrier `bar`, 64 threads).  Then each
+// lane's 16 codes are word (l & 7) of group 8 blk + 4 hf + l / 8.
+template <typename TIn>
+__device__ __forceinline__ void g1_rotate_half(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
+                                               int blk, int hf, int G, uint8_t* act, float* xch, int bar, int lane) {
+  const int64_t e0 = static_cast<int64_t>(blk) * kHB + 512 * hf + 16 * lane;
+  float v[16];
+  load8<TIn>(x + e0, v);
+  load8<TIn>(x + e0 + 8, v + 8);
+  float scale = 1.f;
+  if (signs != nullptr) {
+    const uint4 sg = *reinterpret_cast<const uint4*>(signs + e0);
+    const uint32_t sw[4] = {sg.x, sg.y, sg.z, sg.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t sbit = (sw[i >> 2] << (24 - 8 * (i & 3))) & 0x80000000u;
+      v[i] = __int_as_float(__float_as_int(v[i]) ^ static_cast<int>(sbit));
+    }
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if ((i & h) == 0) {
+          const float a = v[i], b = v[i + h];
+          v[i] = a + b;
+          v[i + h] = a - b;
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const float sgn = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = fmaf(sgn, v[i], __shfl_xor_sync(0xffffffffu, v[i], m));
+    }
+    float4* mine = reinterpret_cast<float4*>(xch + 512 * hf + 16 * lane);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mine[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+    const float4* other = reinterpret_cast<const float4*>(xch + 512 * (1 - hf) + 16 * lane);
+    const float sgn = hf ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 o = other[i];
+      v[4 * i] = fmaf(sgn, v[4 * i], o.x);
+      v[4 * i + 1] = fmaf(sgn, v[4 * i + 1], o.y);
+      v[4 * i + 2] = fmaf(sgn, v[4 * i + 2], o.z);
+      v[4 * i + 3] = fmaf(sgn, v[4 * i + 3], o.w);
+    }
+    scale = kHNorm;
+  }
+  // 16-bit fixed point of the group (8 lanes)
+  float mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  mx *= scale;
+  const float e = mx / kQMax;
+  const float inv = mx > 0.f ? (kQMax / mx) * scale : 0.f;
+  int q[16];
+  int qs = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    q[i] = max(-32512, min(32512, __float2int_rn(v[i] * inv)));
+    qs += q[i];
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+  uint32_t wv[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      wv[2 * j + h] = __byte_perm(static_cast<uint32_t>(q[8 * h + j]), static_cast<uint32_t>(q[8 * h + j + 4]), 0x5410);
+  const int g = blk * 8 + 4 * hf + (lane >> 3);
+  uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupBytes + 32 * (lane & 7));
+  dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+  if ((lane & 7) == 0) {
+    int2 inf;
+    inf.x = __float_as_int(e);
+    inf.y = qs;
+    reinterpret_cast<int2*>(act + G * kG1GroupBytes)[g] = inf;
+  }
+}
+
 // Activation words for long K: one warp per 1024-block, 4 warps per CTA,
 // written to `ws` in the layout above.  Waits for the previous kernel on the
 // stream (which may have produced x, or may still read ws) before touching
@@ -244,27 +330,6 @@ __global__ void __launch_bounds__(128) prep_gemv1_kernel(const TIn* __restrict__
   if (live) g1_rotate_block<TIn>(x, sg, signs != nullptr, blk, K >> 7, ws, lane);
 }
 
-// ---------------------------------------------------------------- prefetch
-// One 32-thread CTA per decode CTA: L2 prefetch of the decode CTA's packed
-// rows and scales (contiguous in memory), then a wait for the previous kernel
-// on the stream, so that the decode kernel's own wait (for this kernel) also
-// covers that one.
-__global__ void __launch_bounds__(32) gemv1_prefetch_kernel(const uint8_t* __restrict__ packed,
-                                                            const uint16_t* __restrict__ scales, int N, int K, int R) {
-  pdl_launch_dependents();
-  if (threadIdx.x == 0) {
-    const int r0 = blockIdx.x * R;
-    const int rows = min(R, N - r0);
-    const int64_t row_bytes = K / 4;
-    const uint8_t* w = packed + static_cast<int64_t>(r0) * row_bytes;
-    const int64_t wbytes = static_cast<int64_t>(rows) * row_bytes;
-    for (int64_t o = 0; o < wbytes; o += kG1PrefetchPiece)
-      prefetch_l2(w + o, static_cast<uint32_t>(wbytes - o < kG1PrefetchPiece ? wbytes - o : kG1PrefetchPiece));
-    prefetch_l2(scales + static_cast<int64_t>(r0) * (K / 128), static_cast<uint32_t>(rows * (K / 128) * 2));
-  }
-  pdl_wait();
-}
-
 // ---------------------------------------------------------------- decode
 // Stage s: its chunks' weight boxes into slot `slot`, completing on `bar`.
 __device__ __forceinline__ void gemv1_issue(const CUtensorMap* tm, const Gemv1Params& p, uint8_t* ring,
@@ -278,24 +343,28 @@ __device__ __forceinline__ void gemv1_issue(const CUtensorMap* tm, const Gemv1Pa
 
 // sum_k c_k q_k of one row's group: 8 packed words against the group's 64
 // activation words (the four T_j combined exactly).
+// One accumulator per slot j (words i = 0..3 and 4..7 in two halves so that
+// each chain is 8 deep); |T_j| <= 16 * 2 * 32512 * 128 < 2^31.
 __device__ __forceinline__ int g1_group_dot(const uint4& wa, const uint4& wb, const uint32_t (&A)[64]) {
   const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-  int lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
+  int t[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t c = w[i] & (0x03030303u << (2 * j));
-      lo[j] = dp2a_lo(A[8 * i + 2 * j], c, lo[j]);
-      hi[j] = dp2a_hi(A[8 * i + 2 * j + 1], c, hi[j]);
+      int& acc = t[i >> 2][j];
+      acc = dp2a_lo(A[8 * i + 2 * j], c, acc);
+      acc = dp2a_hi(A[8 * i + 2 * j + 1], c, acc);
     }
   }
-  return (lo[0] + hi[0]) + ((lo[1] + hi[1]) >> 2) + ((lo[2] + hi[2]) >> 4) + ((lo[3] + hi[3]) >> 6);
+  return (t[0][0] + t[1][0]) + ((t[0][1] + t[1][1]) >> 2) + ((t[0][2] + t[1][2]) >> 4) +
+         ((t[0][3] + t[1][3]) >> 6);
 }
 
 // TPW: row tiles per warp at most (1, 2 or 4).
 template <typename TIn, typename TOut, bool kFused, int TPW>
-__global__ void __maxnreg__(kG1MaxRegs)
+__global__ void __launch_bounds__(kG1Threads, 2)
     gemv1_2bit_kernel(const __grid_constant__ CUtensorMap tm_w, const Gemv1Params p) {
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
@@ -348,16 +417,28 @@ __global__ void __maxnreg__(kG1MaxRegs)
   }
   if constexpr (kFused) {
     const int nblk = p.K >> 10;
-    uint32_t sg0[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sg1[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const bool b0 = warp < nblk, b1 = warp + kG1Warps < nblk;
-    if (p.signs != nullptr) {
-      if (b0) g1_load_signs(p.signs, warp, lane, sg0);
-      if (b1) g1_load_signs(p.signs, warp + kG1Warps, lane, sg1);
-    }
-    pdl_wait();  // x may be the previous kernel's output
     const TIn* x = static_cast<const TIn*>(p.x);
-    if (b0) g1_rotate_block<TIn>(x, sg0, p.signs != nullptr, warp, G, act, lane);
-    if (b1) g1_rotate_block<TIn>(x, sg1, p.signs != nullptr, warp + kG1Warps, G, act, lane);
+    if (g1_half_blocks(p.K)) {
+      pdl_wait();  // x may be the previous kernel's output
+      if (warp < 2 * nblk)
+        g1_rotate_half<TIn>(x, p.signs, warp >> 1, warp & 1, G, act, red + (warp >> 1) * kHB, 1 + (warp >> 1), lane);
+    } else {
+      // blocks warp, warp + 8, warp + 16; the first two blocks' signs are
+      // loaded before the wait
+      uint32_t sg0[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sg1[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      const bool b0 = warp < nblk, b1 = warp + kG1Warps < nblk, b2 = warp + 2 * kG1Warps < nblk;
+      if (p.signs != nullptr) {
+        if (b0) g1_load_signs(p.signs, warp, lane, sg0);
+        if (b1) g1_load_signs(p.signs, warp + kG1Warps, lane, sg1);
+      }
+      pdl_wait();  // x may be the previous kernel's output
+      if (b0) g1_rotate_block<TIn>(x, sg0, p.signs != nullptr, warp, G, act, lane);
+      if (b1) g1_rotate_block<TIn>(x, sg1, p.signs != nullptr, warp + kG1Warps, G, act, lane);
+      if (b2) {
+        if (p.signs != nullptr) g1_load_signs(p.signs, warp + 2 * kG1Warps, lane, sg0);
+        g1_rotate_block<TIn>(x, sg0, p.signs != nullptr, warp + 2 * kG1Warps, G, act, lane);
+      }
+    }
   }
   __syncthreads();
 
@@ -366,74 +447,77 @@ __global__ void __maxnreg__(kG1MaxRegs)
   const bool active = tg < p.Wt;
   const int t0 = tg * p.RT / p.Wt, nt = active ? (tg + 1) * p.RT / p.Wt - t0 : 0;  // this warp's row tiles
   const int2* info = reinterpret_cast<const int2*>(act + G * kG1GroupBytes);
-  // byte offsets of the lane's rows in a box (the group's two 16-byte pieces
-  // 2 gslot, 2 gslot + 1, swizzled with the row index mod 8 = rsub) and of
-  // the rows' scales; rows past the CTA's end read valid rows, sums dropped
-  const int u0 = ((2 * gslot) ^ rsub) << 4, u1 = ((2 * gslot + 1) ^ rsub) << 4;
-  int roff[TPW], soff[TPW];
+  // byte offsets in a box of the lane's two 16-byte pieces (2 gslot and
+  // 2 gslot + 1 of the row's 128 bytes, swizzled with the row index mod 8 =
+  // rsub) and of the rows' scales; rows past the CTA's end read valid rows
+  // and their sums are dropped
+  const int u0 = ((2 * gslot) ^ rsub) << 4;
+  int pa[TPW], soff[TPW];
   float acc[TPW];
 #pragma unroll
   for (int i = 0; i < TPW; ++i) {
     const int r = 8 * (t0 + i) + rsub;
-    roff[i] = min(r, p.R - 1) * 128;
+    pa[i] = min(r, p.R - 1) * 128 + u0;
     soff[i] = min(r, nrows - 1) * G;
     acc[i] = 0.f;
   }
+  const bool refill = p.nslots < p.nstage;
 
   bool ok = __all_sync(0xffffffffu, mbar_wait_backoff(pre_bar, 0, FAULT_WAIT_ACT));
-  int c = active ? wk : C;  // this warp's next chunk
-  for (int s = 0; s < p.nstage && ok; ++s) {
-    const int cend = min(C, (s + 1) * p.NB);
-    if (c < cend) {
+  int cur_s = -1;
+  const uint8_t* sbase = ring;  // slot of the current stage
+  for (int c = active && ok ? wk : C; c < C; c += p.Wk) {
+    const int s = c >> p.nb_log2;
+    if (s != cur_s) {
       ok = __all_sync(0xffffffffu, mbar_wait_backoff(&full[s], 0, FAULT_WAIT_FULL)) &&
            *reinterpret_cast<volatile uint32_t*>(cta_fault) == 0u;
       if (!ok) break;
-      const uint8_t* slot = ring + static_cast<int64_t>(s % p.nslots) * p.slot_bytes;
-      const int cbeg = s * p.NB;
-      for (; c < cend; c += p.Wk) {
-        const int g = 4 * c + gslot;
-        uint32_t A[64];
-        const uint4* src = reinterpret_cast<const uint4*>(act + g * kG1GroupBytes);
+      cur_s = s;
+      sbase = ring + static_cast<int64_t>(s % p.nslots) * p.slot_bytes;
+    }
+    const uint8_t* box = sbase + (c - (s << p.nb_log2)) * p.box_stride;
+    const int g = 4 * c + gslot;
+    uint32_t A[64];
+    const uint4* src = reinterpret_cast<const uint4*>(act + g * kG1GroupBytes);
 #pragma unroll
-        for (int v = 0; v < 16; ++v) {
-          const uint4 u4 = src[v];
-          A[4 * v] = u4.x;
-          A[4 * v + 1] = u4.y;
-          A[4 * v + 2] = u4.z;
-          A[4 * v + 3] = u4.w;
-        }
-        const int2 inf = info[g];
-        const float e = __int_as_float(inf.x);
-        const uint8_t* box = slot + (c - cbeg) * p.box_stride;
-        if constexpr (TPW == 1) {
-          const uint4 w0 = *reinterpret_cast<const uint4*>(box + roff[0] + u0);
-          const uint4 w1 = *reinterpret_cast<const uint4*>(box + roff[0] + u1);
-          const float sa = __half2float(sc[soff[0] + g]) * e;
-          acc[0] = fmaf(__int2float_rn(g1_group_dot(w0, w1, A) - inf.y), sa, acc[0]);
-        } else {
+    for (int v = 0; v < 16; ++v) {
+      const uint4 u4 = src[v];
+      A[4 * v] = u4.x;
+      A[4 * v + 1] = u4.y;
+      A[4 * v + 2] = u4.z;
+      A[4 * v + 3] = u4.w;
+    }
+    const int2 inf = info[g];
+    const float e = __int_as_float(inf.x);
+    if constexpr (TPW == 1) {
+      const uint4 w0 = *reinterpret_cast<const uint4*>(box + pa[0]);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(box + (pa[0] ^ 16));
+      const float sa = __half2float(sc[soff[0] + g]) * e;
+      acc[0] = fmaf(__int2float_rn(g1_group_dot(w0, w1, A) - inf.y), sa, acc[0]);
+    } else {
 #pragma unroll
-          for (int tp = 0; tp < TPW; tp += 2) {
-            // tiles beyond nt compute on valid rows and are dropped at the end
-            const uint4 wa0 = *reinterpret_cast<const uint4*>(box + roff[tp] + u0);
-            const uint4 wa1 = *reinterpret_cast<const uint4*>(box + roff[tp] + u1);
-            const uint4 wb0 = *reinterpret_cast<const uint4*>(box + roff[tp + 1] + u0);
-            const uint4 wb1 = *reinterpret_cast<const uint4*>(box + roff[tp + 1] + u1);
-            const float sa = __half2float(sc[soff[tp] + g]) * e;
-            const float sb = __half2float(sc[soff[tp + 1] + g]) * e;
-            const int da = g1_group_dot(wa0, wa1, A) - inf.y;
-            const int db = g1_group_dot(wb0, wb1, A) - inf.y;
-            acc[tp] = fmaf(__int2float_rn(da), sa, acc[tp]);
-            acc[tp + 1] = fmaf(__int2float_rn(db), sb, acc[tp + 1]);
-          }
-        }
+      for (int tp = 0; tp < TPW; tp += 2) {
+        // tiles beyond nt compute on valid rows and are dropped at the end
+        const uint4 wa0 = *reinterpret_cast<const uint4*>(box + pa[tp]);
+        const uint4 wa1 = *reinterpret_cast<const uint4*>(box + (pa[tp] ^ 16));
+        const uint4 wb0 = *reinterpret_cast<const uint4*>(box + pa[tp + 1]);
+        const uint4 wb1 = *reinterpret_cast<const uint4*>(box + (pa[tp + 1] ^ 16));
+        const float sa = __half2float(sc[soff[tp] + g]) * e;
+        const float sb = __half2float(sc[soff[tp + 1] + g]) * e;
+        const int da = g1_group_dot(wa0, wa1, A) - inf.y;
+        const int db = g1_group_dot(wb0, wb1, A) - inf.y;
+        acc[tp] = fmaf(__int2float_rn(da), sa, acc[tp]);
+        acc[tp + 1] = fmaf(__int2float_rn(db), sb, acc[tp + 1]);
       }
     }
-    // the warp completing stage s refills its slot with stage s + nslots
-    if (p.nslots < p.nstage) {
+    if (refill) {
+      // a stage's chunks are each used by Wt warps; the last use refills the
+      // slot with the stage nslots ahead
       __syncwarp();
       if (lane == 0) {
         __threadfence_block();
-        if (atomicAdd(&done[s], 1u) == static_cast<uint32_t>(kG1Warps - 1) && s + p.nslots < p.nstage) {
+        const int nch = min(p.NB, C - (s << p.nb_log2));
+        if (atomicAdd(&done[s], 1u) == static_cast<uint32_t>(nch * p.Wt - 1) && s + p.nslots < p.nstage) {
           __threadfence_block();
           issued[s + p.nslots] = 1u;
           gemv1_issue(&tm_w, p, ring, &full[s + p.nslots], s + p.nslots, s % p.nslots, r0);

@@ -278,7 +278,7 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, Gemv
 }
 
 struct G1Plan {
-  int grid, R, RT, Wt, Wk, TPW, NB, nstage, nslots, box_stride, slot_bytes;
+  int grid, R, RT, Wt, Wk, TPW, NB, nb_log2, nstage, nslots, box_stride, slot_bytes;
   bool fused;
   Gemv1Layout lay;
 };
@@ -315,9 +315,15 @@ bool g1_plan(int64_t N, int64_t K, int sm_count, int max_smem, bool fused, G1Pla
   if (best_cost < 0) return false;
   pl.box_stride = static_cast<int>(align_up(R * 128, 1024));
   // stages of at least 8 KB of weights
-  int64_t nb = (8192 + R * 128 - 1) / (R * 128);
-  if (nb > C) nb = C;
-  if (nb < 1) nb = 1;
+  // stages of at least 8 KB of weights, a power of two of chunks
+  int64_t want = (8192 + R * 128 - 1) / (R * 128);
+  if (want > C) want = C;
+  int64_t nb = 1;
+  pl.nb_log2 = 0;
+  while (nb < want) {
+    nb *= 2;
+    ++pl.nb_log2;
+  }
   pl.NB = static_cast<int>(nb);
   pl.nstage = static_cast<int>((C + nb - 1) / nb);
   pl.slot_bytes = static_cast<int>(nb) * pl.box_stride;
@@ -491,9 +497,8 @@ tb_status launch_gemv(const LinearArgs& a, const DevInfo* d, const GemvPlan& pl,
   return launch_pdl(k, dim3(pl.grid), dim3(kGemvThreads), pl.smem, a.st, tm, p);
 }
 
-// One token: gemv1_prefetch_kernel, then gemv1_2bit_kernel, with the rotation
-// inside the decode kernel for K up to kG1FusedMaxBlocks 1024-blocks, else
-// prep_gemv1_kernel before it.
+// One token: gemv1_2bit_kernel, with the rotation inside it for K up to
+// kG1FusedMaxBlocks 1024-blocks, else after prep_gemv1_kernel.
 template <typename TIn, typename TOut, bool kFused>
 tb_status launch_gemv1(const LinearArgs& a, const DevInfo* d, const G1Plan& pl, const CUtensorMap& tm,
                        const Gemv1Params& p) {
@@ -528,6 +533,7 @@ tb_status run_gemv1_typed(const LinearArgs& a, const DevInfo* d, const G1Plan& p
   p.Wt = pl.Wt;
   p.Wk = pl.Wk;
   p.NB = pl.NB;
+  p.nb_log2 = pl.nb_log2;
   p.nstage = pl.nstage;
   p.nslots = pl.nslots;
   p.box_stride = pl.box_stride;
@@ -536,9 +542,6 @@ tb_status run_gemv1_typed(const LinearArgs& a, const DevInfo* d, const G1Plan& p
   p.off_sc = pl.lay.off_sc;
   p.off_red = pl.lay.off_red;
   p.off_bar = pl.lay.off_bar;
-  if (launch_pdl(gemv1_prefetch_kernel, dim3(pl.grid), dim3(32), 0, a.st, a.packed, a.scales, p.N, p.K, p.R) !=
-      TB_OK)
-    return TB_ERR_CUDA;
   if (!pl.fused) {
     const dim3 pgrid(static_cast<unsigned>((a.K / kHB + 3) / 4));
     if (launch_pdl(prep_gemv1_kernel<TIn>, pgrid, dim3(128), 0, a.st, static_cast<const TIn*>(a.x), a.signs,
