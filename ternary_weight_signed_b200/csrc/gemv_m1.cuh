@@ -65,8 +65,9 @@ constexpr int kG1Threads = 32 * kG1Warps;
 // Shared memory per CTA for two CTAs per SM (228 KB per SM, 1 KB reserved per CTA).
 constexpr int kG1SmemMax = 115 * 1024 - 2048;
 constexpr int kG1MaxRows = 256;  // TMA box height limit
-// The CTA rotates x itself for K up to this many 1024-blocks (three per warp).
-constexpr int kG1FusedMaxBlocks = 3 * kG1Warps;
+// The CTA rotates x itself for K up to this many 1024-blocks (one per warp);
+// longer K goes through prep_gemv1_kernel.
+constexpr int kG1FusedMaxBlocks = kG1Warps;
 constexpr int kG1GroupBytes = 256;
 
 // d = c + a.lo16 * b.byte0 + a.hi16 * b.byte1 (lo) or * bytes 2, 3 (hi);
@@ -423,21 +424,13 @@ __global__ void __launch_bounds__(kG1Threads, 2)
       if (warp < 2 * nblk)
         g1_rotate_half<TIn>(x, p.signs, warp >> 1, warp & 1, G, act, red + (warp >> 1) * kHB, 1 + (warp >> 1), lane);
     } else {
-      // blocks warp, warp + 8, warp + 16; the first two blocks' signs are
-      // loaded before the wait
-      uint32_t sg0[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sg1[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      const bool b0 = warp < nblk, b1 = warp + kG1Warps < nblk, b2 = warp + 2 * kG1Warps < nblk;
-      if (p.signs != nullptr) {
-        if (b0) g1_load_signs(p.signs, warp, lane, sg0);
-        if (b1) g1_load_signs(p.signs, warp + kG1Warps, lane, sg1);
-      }
+      // block `warp` (K <= kG1FusedMaxBlocks blocks); its signs are loaded
+      // before the wait
+      uint32_t sg[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      const bool live = warp < nblk;
+      if (live && p.signs != nullptr) g1_load_signs(p.signs, warp, lane, sg);
       pdl_wait();  // x may be the previous kernel's output
-      if (b0) g1_rotate_block<TIn>(x, sg0, p.signs != nullptr, warp, G, act, lane);
-      if (b1) g1_rotate_block<TIn>(x, sg1, p.signs != nullptr, warp + kG1Warps, G, act, lane);
-      if (b2) {
-        if (p.signs != nullptr) g1_load_signs(p.signs, warp + 2 * kG1Warps, lane, sg0);
-        g1_rotate_block<TIn>(x, sg0, p.signs != nullptr, warp + 2 * kG1Warps, G, act, lane);
-      }
+      if (live) g1_rotate_block<TIn>(x, sg, p.signs != nullptr, warp, G, act, lane);
     }
   }
   __syncthreads();
