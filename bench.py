@@ -136,10 +136,10 @@ def _traffic(fmt):
 # ---------------------------------------------------------------------------- ours
 def _launches_per_call(tb, fmt, m, n, k):
     """Kernels one tb_ternary_linear call launches on the path it takes: the
-    one-token 2-bit decode kernel rotates x itself up to K = 24576 (one launch);
+    one-token 2-bit decode kernel rotates x itself up to K = 8192 (one launch);
     the other float paths run an activation prep kernel and one main kernel."""
     path = tb.tb_ternary_linear_path(tb.TB_BF16, fmt, m, n, k, True, True)
-    if path == tb.TB_PATH_GEMV and fmt == "2bit" and m == 1 and k // 1024 <= 24:
+    if path == tb.TB_PATH_GEMV and fmt == "2bit" and m == 1 and k // 1024 <= 8:
         return 1
     if path == tb.TB_PATH_GEMV and fmt == "base3":
         return 2 * ((m + 3) // 4)

@@ -342,6 +342,14 @@ bool g1_plan(int64_t N, int64_t K, int sm_count, int max_smem, bool fused, G1Pla
 
 bool g1_fused(int64_t K) { return K / kHB <= kG1FusedMaxBlocks; }
 
+// The two-CTA one-token kernel wins when it rotates x itself or has at least
+// eight row tiles per CTA; with few rows and long K (a down projection,
+// 5120 x 17408: 19.3 against 23.3 us per call on B200) the 16-warp kernel with
+// dynamic item distribution is faster.
+bool g1_preferred(int64_t N, int64_t K, int sm_count) {
+  return g1_fused(K) || (N + sm_count - 1) / sm_count >= 64;
+}
+
 struct B3Plan {
   int grid, R, RT, NB, nstage, nslots, box_stride, slot_bytes, sc_bytes;
   size_t smem;
@@ -451,7 +459,7 @@ bool gemv_ok(const LinearArgs& a) {
     B3Plan pl;
     return b3_plan(std::min<int64_t>(a.M, kGemvMaxM), a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
   }
-  if (a.M == 1) {
+  if (a.M == 1 && g1_preferred(a.N, a.K, kB200Sms)) {
     G1Plan p1;
     if (g1_plan(a.N, a.K, kB200Sms, kB200SmemOptin, g1_fused(a.K), &p1)) return true;
   }
@@ -556,7 +564,7 @@ tb_status run_gemv1_typed(const LinearArgs& a, const DevInfo* d, const G1Plan& p
 
 template <typename TIn>
 tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
-  if (a.M == 1) {
+  if (a.M == 1 && g1_preferred(a.N, a.K, d->sm_count)) {
     G1Plan p1;
     if (g1_plan(a.N, a.K, d->sm_count, d->max_smem_optin, g1_fused(a.K), &p1)) return run_gemv1_typed<TIn>(a, d, p1);
   }
