@@ -8,9 +8,10 @@
 //   B = fp16(s * t), which is exact because t is -1, 0 or +1 and s is an fp16
 //       value, so no per-group rescaling of the accumulator is needed.
 //
-// Tile: 256 tokens x 256 weight rows, K in stages of 64 (one 128-byte swizzle
-// atom of fp16).  The 256 tokens are two M=128 MMAs that share the unpacked B
-// tile, each with its own 128 x 256 fp32 accumulator (all 512 TMEM columns).
+// Tile: 256 tokens x BN weight rows (BN = 128, 192 or 256, chosen per shape
+// so that the tiles fill whole waves of SMs), K in stages of 64 (one 128-byte
+// swizzle atom of fp16).  The 256 tokens are two M=128 MMAs that share the
+// unpacked B tile, each with its own 128 x BN fp32 accumulator in TMEM.
 // Warp roles:
 //   warp 0    : TMA producer (x' tile with 128B swizzle, packed 2-bit codes);
 //   warp 1    : TMEM allocation and the single thread issuing tcgen05.mma;
@@ -39,23 +40,28 @@ namespace tb {
 
 constexpr int kGemmBM = 256;      // tokens per tile: two MMAs of M = 128
 constexpr int kGemmUM = 128;      // M of one MMA (TMEM lanes)
-constexpr int kGemmBN = 256;
+constexpr int kGemmBN = 256;     // widest weight tile
 constexpr int kGemmBK = 64;
 constexpr int kGemmStages = 3;
 constexpr int kGemmUnpackWarps = 8;
 constexpr int kGemmThreads = 32 * (2 + kGemmUnpackWarps);
 constexpr int kGemmTmemCols = 512;
 constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 32 KB
-constexpr int kGemmBBytes = kGemmBN * kGemmBK * 2;  // 32 KB
-constexpr int kGemmWBytes = kGemmBN * kGemmBK / 4;  // 4 KB of packed codes
-constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes + kGemmWBytes;
-constexpr int kGemmSmemBytes = kGemmStages * kGemmStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+// per weight-tile width BN: B (fp16 s*t) and the packed codes of a stage
+__host__ __device__ constexpr int gemm_b_bytes(int bn) { return bn * kGemmBK * 2; }
+__host__ __device__ constexpr int gemm_w_bytes(int bn) { return bn * kGemmBK / 4; }
+__host__ __device__ constexpr int gemm_stage_bytes(int bn) { return kGemmABytes + gemm_b_bytes(bn) + gemm_w_bytes(bn); }
+__host__ __device__ constexpr int gemm_smem_bytes(int bn) {
+  return kGemmStages * gemm_stage_bytes(bn) + 1024 /*align*/ + 256 /*barriers*/;
+}
+constexpr int kGemmSmemBytes = gemm_smem_bytes(kGemmBN);
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B fp16
 // (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
 // M >> 4 at bits 24-28.
-constexpr uint32_t kGemmIdesc =
-    (1u << 4) | (static_cast<uint32_t>(kGemmBN >> 3) << 17) | (static_cast<uint32_t>(kGemmUM >> 4) << 24);
+__host__ __device__ constexpr uint32_t gemm_idesc(int bn) {
+  return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(kGemmUM >> 4) << 24);
+}
 
 // Shared-memory matrix descriptor for a K-major operand in the canonical
 // 128-byte swizzled layout: rows of 128 bytes, 8-row groups 1024 bytes apart
@@ -191,20 +197,23 @@ __device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, c
   }
 }
 
-template <typename TOut>
+template <int BN, typename TOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_2bit_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                         const GemmParams p) {
+  static_assert(BN % 32 == 0 && BN >= 128 && BN <= kGemmBN, "weight tile width");
+  constexpr int kStage = gemm_stage_bytes(BN), kB = gemm_b_bytes(BN), kW = gemm_w_bytes(BN);
+  constexpr uint32_t kIdesc = gemm_idesc(BN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmStages * kGemmStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmStages * kStage);
   uint64_t* bready = full + kGemmStages;
   uint64_t* empty = bready + kGemmStages;
   uint64_t* accum = empty + kGemmStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kGemmBN, m0 = blockIdx.y * kGemmBM;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kGemmBM;
   const int nk = p.K / kGemmBK;
 
   if (threadIdx.x == 0) {
@@ -236,10 +245,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (kb >= kGemmStages &&
             !mbar_wait(&empty[s], ((kb / kGemmStages) & 1) ^ 1, FAULT_WAIT_EMPTY))
           break;
-        uint8_t* st = smem + s * kGemmStageBytes;
-        mbar_arrive_expect_tx(&full[s], kGemmABytes + kGemmWBytes);
+        uint8_t* st = smem + s * kStage;
+        mbar_arrive_expect_tx(&full[s], kGemmABytes + kW);
         tma_load_2d(st, &tm_x, kb * kGemmBK, m0, &full[s]);
-        tma_load_2d(st + kGemmABytes + kGemmBBytes, &tm_w, kb * (kGemmBK / 16), n0, &full[s]);
+        tma_load_2d(st + kGemmABytes + kB, &tm_w, kb * (kGemmBK / 16), n0, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -252,14 +261,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ok = mbar_wait(&full[s], par, FAULT_WAIT_FULL) && mbar_wait(&bready[s], par, FAULT_WAIT_FULL);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + s * kGemmStageBytes);
+        const uint32_t a = smem_u32(smem + s * kStage);
         const uint32_t b = a + kGemmABytes;
 #pragma unroll
         for (int kk = 0; kk < kGemmBK / 16; ++kk) {
           const uint64_t bd = umma_desc_sw128(b + 32 * kk);
           const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-          umma_f16(tmem, umma_desc_sw128(a + 32 * kk), bd, kGemmIdesc, acc);
-          umma_f16(tmem + kGemmBN, umma_desc_sw128(a + kGemmUM * 128 + 32 * kk), bd, kGemmIdesc, acc);
+          umma_f16(tmem, umma_desc_sw128(a + 32 * kk), bd, kIdesc, acc);
+          umma_f16(tmem + BN, umma_desc_sw128(a + kGemmUM * 128 + 32 * kk), bd, kIdesc, acc);
         }
         umma_commit(&empty[s]);
       }
@@ -268,9 +277,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ---------------------------------------------------------------- unpack
     const int r = threadIdx.x - 64;  // weight row of the tile this thread unpacks (0..255)
+    const bool in_tile = r < BN;     // threads past the tile width only take part in the barriers
     const int G = p.K / 128;
     const int n = n0 + r;
-    const bool row_ok = n < p.N;
+    const bool row_ok = in_tile && n < p.N;
     const uint16_t* srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
     __half s_next = __ushort_as_half(row_ok ? srow[0] : uint16_t(0));
     __half s_cur = s_next;
@@ -291,13 +301,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         s_cur = s_next;
         if (g + 1 < G) s_next = __ushort_as_half(row_ok ? srow[g + 1] : uint16_t(0));
       }
-      uint8_t* st = smem + s * kGemmStageBytes;
-      const uint4 w4 = *reinterpret_cast<const uint4*>(st + kGemmABytes + kGemmBBytes + r * 16);
+      uint8_t* st = smem + s * kStage;
+      const uint4 w4 = in_tile ? *reinterpret_cast<const uint4*>(st + kGemmABytes + kB + r * 16) : make_uint4(0, 0, 0, 0);
       const __half2 s2 = __halves2half2(s_cur, s_cur);
       const __half2 ns2 = __hneg2(s2);
       uint8_t* row = st + kGemmABytes + r * 128;
 #pragma unroll
-      for (int wd = 0; wd < 4; ++wd) {
+      for (int wd = 0; wd < 4 && in_tile; ++wd) {
         const uint32_t w = (&w4.x)[wd];
         uint32_t o[8];
 #pragma unroll
@@ -328,9 +338,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       TOut* y = reinterpret_cast<TOut*>(p.y);
       const bool vec = (p.N % static_cast<int>(16 / sizeof(TOut))) == 0;  // 16-byte row alignment
 #pragma unroll 1
-      for (int c = 0; c < kGemmBN / 32; ++c) {
+      for (int c = 0; c < BN / 32; ++c) {
         uint32_t v32[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(kGemmBN * h + 32 * c), v32);
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(BN * h + 32 * c), v32);
         tmem_ld_wait();
         const int nb = n0 + 32 * c;
         if (m < p.M && nb < p.N) {

@@ -339,7 +339,8 @@ __device__ __forceinline__ void gemv1_issue(const CUtensorMap* tm, const Gemv1Pa
   const int nb = min(p.NB, C - s * p.NB);
   uint8_t* dst = ring + static_cast<int64_t>(slot) * p.slot_bytes;
   mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb) * static_cast<uint32_t>(p.R) * 128u);
-  for (int b = 0; b < nb; ++b) tma_load_2d(dst + b * p.box_stride, tm, (s * p.NB + b) * 128, r0, bar);
+  const uint64_t pol = l2_policy_evict_first();  // weights are read once per call
+  for (int b = 0; b < nb; ++b) tma_load_2d_hint(dst + b * p.box_stride, tm, (s * p.NB + b) * 128, r0, bar, pol);
 }
 
 // sum_k c_k q_k of one row's group: 8 packed words against the group's 64

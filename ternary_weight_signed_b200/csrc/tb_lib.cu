@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <unordered_set>
 
@@ -840,12 +841,31 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
     default: launch_prep_gemm<float>(a, xh); break;
   }
   if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  // Weight-tile width: wave fill of the SMs times the tile's own efficiency.
+  // Narrower tiles reuse each activation stage for fewer weight rows and leave
+  // unpack warps idle; on B200 the 192-wide tile ran the prefill shape
+  // (2048 x 17408 x 5120) at 0.90 of the 256-wide tile's per-tile rate, which
+  // its better wave fill (4.92 against 3.68 waves) does not make up.
+  const int64_t mt = (a.M + kGemmBM - 1) / kGemmBM;
+  int bn = 256;
+  double best = -1.0;
+  const int cands[3] = {256, 192, 128};
+  const double eff[3] = {1.0, 0.9, 0.8};
+  for (int i = 0; i < 3; ++i) {
+    const double tiles = static_cast<double>(((a.N + cands[i] - 1) / cands[i]) * mt);
+    const double waves = tiles / d->sm_count;
+    const double score = eff[i] * waves / std::ceil(waves);
+    if (score > best + 1e-9) {
+      best = score;
+      bn = cands[i];
+    }
+  }
   CUtensorMap tm_x, tm_w;
   if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGemmBK, kGemmBM,
                   CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
   if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, kGemmBK / 16,
-                  kGemmBN) != TB_OK)
+                  static_cast<uint32_t>(bn)) != TB_OK)
     return TB_ERR_CUDA;
   GemmParams gp;
   gp.M = static_cast<int>(a.M);
@@ -853,16 +873,23 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   gp.K = static_cast<int>(a.K);
   gp.y = a.y;
   gp.scales = a.scales;
-  const dim3 grid(static_cast<unsigned>((a.N + kGemmBN - 1) / kGemmBN),
-                  static_cast<unsigned>((a.M + kGemmBM - 1) / kGemmBM));
-  if (a.yt == TB_FP32) {
-    auto k = gemm_2bit_tc_kernel<float>;
-    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
-    return launch_pdl(k, grid, dim3(kGemmThreads), kGemmSmemBytes, a.st, tm_x, tm_w, gp);
+  const dim3 grid(static_cast<unsigned>((a.N + bn - 1) / bn), static_cast<unsigned>(mt));
+#define TB_GEMM_LAUNCH(BN)                                                                                   \
+  if (bn == BN) {                                                                                            \
+    if (a.yt == TB_FP32) {                                                                                   \
+      auto k = gemm_2bit_tc_kernel<BN, float>;                                                               \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
+      return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BN)), a.st, tm_x, tm_w, gp); \
+    }                                                                                                        \
+    auto k = gemm_2bit_tc_kernel<BN, __nv_bfloat16>;                                                         \
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                       \
+    return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BN)), a.st, tm_x, tm_w, gp);   \
   }
-  auto k = gemm_2bit_tc_kernel<__nv_bfloat16>;
-  if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;
-  return launch_pdl(k, grid, dim3(kGemmThreads), kGemmSmemBytes, a.st, tm_x, tm_w, gp);
+  TB_GEMM_LAUNCH(256)
+  TB_GEMM_LAUNCH(192)
+  TB_GEMM_LAUNCH(128)
+#undef TB_GEMM_LAUNCH
+  return TB_ERR_SHAPE;
 }
 
 tb_status validate_linear(const LinearArgs& a) {

@@ -62,6 +62,9 @@ WORKLOAD_CASES = [
     (11, 2, 6144, 6144, 0.2, "abs_normal", 0.0),       # q-projection shape
     (12, 1, 1024, 3072, 0.5, "abs_normal", 0.0),       # K/512 not a multiple of the stage width
     (13, 3, 5120, 6144, 0.33, "abs_normal", 0.01),     # o-projection shape
+    (14, 2, 17408, 5120, 0.33, "abs_normal", 0.01),    # gate/up, two tokens (two-CTA decode kernel)
+    (15, 4, 17408, 5120, 0.33, "abs_normal", 0.0),     # gate/up, four tokens
+    (16, 3, 9999, 3072, 0.5, "abs_normal", 0.0),       # three tokens in a four-token kernel, ragged N
 ]
 
 
