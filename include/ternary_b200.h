@@ -94,17 +94,18 @@ typedef int tb_dtype;
 typedef int tb_path;
 #define TB_PATH_AUTO 0   /* choose by shape (what tb_ternary_linear does)       */
 #define TB_PATH_GEMV 1   /* CUDA-core streaming kernels on 16-bit fixed-point
-                            activations, for M <= 4 (base-3: M <= 16).  One token
-                            (2-bit): an L2-prefetch launch, then the decode
-                            kernel, which rotates x itself for K <= 32768      */
+                            activations, for M <= 4 (base-3: M <= 7, in chunks
+                            of 4 tokens).  One token (2-bit): one launch that
+                            rotates x itself for K <= 8192                     */
 #define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
                             s*t in shared memory, fp32 accumulators in TMEM)    */
 #define TB_PATH_SIMPLE 3 /* plain per-row kernel: any K % 128, any alignment    */
 #define TB_PATH_GEMV_TC 4 /* tcgen05 decode kernel (codes unpacked into TMEM as
                             the u8 A operand, int8 activation planes as B in
-                            shared memory), for M <= 4 and N <= 148 * 128; same
-                            other rules as TB_PATH_GEMV, slower than it on B200,
-                            never chosen by TB_PATH_AUTO                         */
+                            shared memory), for M <= 16 and N <= 148 * 128;
+                            base-3 with 8-16 tokens is first re-encoded to 2-bit
+                            slots in the workspace.  Chosen by TB_PATH_AUTO from
+                            4 tokens (2-bit) or 8 tokens (base-3)               */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* tb_status_string(tb_status st);

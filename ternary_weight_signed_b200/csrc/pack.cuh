@@ -129,40 +129,68 @@ __global__ void unpack_base3_kernel(const uint16_t* __restrict__ in, int4* __res
   count_invalid(bad, counter);
 }
 
-// Base-3 groups (26 bytes) -> 2-bit slot groups (32 bytes), one thread per
-// group: the prefill GEMM consumes the 2-bit layout, so a base-3 matrix is
-// re-encoded into the caller's workspace first.  Invalid bytes decode as t = 0
-// (as tb_unpack_ternary does; the linear paths leave their output unspecified).
-__global__ void transcode_b3_to_2bit_kernel(const uint16_t* __restrict__ in, uint4* __restrict__ out,
-                                            int64_t ngroups) {
-  const int64_t gi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (gi >= ngroups) return;
-  const uint16_t* p = in + gi * 13;
-  uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-  for (int h = 0; h < 13; ++h) {
-    const uint32_t pair = p[h];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int byte_idx = 2 * h + e;
-      const uint32_t raw = (pair >> (8 * e)) & 0xffu;
-      uint32_t v = raw, dig[5];
+// Base-3 groups (26 bytes) -> 2-bit slot groups (32 bytes): the 2-bit paths
+// (prefill GEMM, tensor-core decode) consume the 2-bit layout, so a base-3
+// matrix is re-encoded into the caller's workspace first.  A warp copies its
+// 32 groups' bytes into shared memory with coalesced loads; then each lane
+// decodes one group through a 243-entry table (byte value -> its five digits,
+// which are the biased codes, as five 2-bit fields) and places each byte's ten
+// bits at bit 10 i of the group's 256-bit slot string.  Invalid bytes decode
+// as t = 0 (as tb_unpack_ternary does; the linear paths leave their output
+// unspecified).  256 threads per block, 256 groups per block.
+__global__ void __launch_bounds__(256) transcode_b3_to_2bit_kernel(const uint8_t* __restrict__ in,
+                                                                   uint4* __restrict__ out, int64_t ngroups) {
+  __shared__ uint16_t lut[256];
+  __shared__ __align__(16) uint8_t buf[8][32 * 26];
+  {
+    const uint32_t i = threadIdx.x;
+    uint32_t code = 0x155u;  // five codes 1 (t = 0)
+    if (i < 243u) {
+      uint32_t v = i;
+      code = 0;
 #pragma unroll
       for (int j = 0; j < 5; ++j) {
-        dig[j] = v % 3u;
+        code |= (v % 3u) << (2 * j);
         v /= 3u;
       }
-      bool invalid = raw >= 243u;
-      if (byte_idx == 25) invalid = invalid || dig[3] != 1u || dig[4] != 1u;
-#pragma unroll
-      for (int j = 0; j < 5; ++j) {
-        const int k = 5 * byte_idx + j;  // code index in the group
-        if (k < 128) w[k >> 4] |= (invalid ? 1u : dig[j]) << (2 * (k & 15));
-      }
     }
+    lut[i] = static_cast<uint16_t>(code);
   }
-  out[2 * gi] = make_uint4(w[0], w[1], w[2], w[3]);
-  out[2 * gi + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t g0 = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * 32;
+  const int64_t left = ngroups - g0;
+  const int ng = left <= 0 ? 0 : (left < 32 ? static_cast<int>(left) : 32);
+  // even; the source is 4-byte aligned: the paths that re-encode need 16-byte
+  // aligned packed weights, and a warp starts at byte 26 * 32 * k
+  const int nbytes = 26 * ng;
+  const uint8_t* src = in + 26 * g0;
+  uint8_t* b = buf[warp];
+  for (int w = lane; w < nbytes / 4; w += 32)
+    reinterpret_cast<uint32_t*>(b)[w] = reinterpret_cast<const uint32_t*>(src)[w];
+  if ((nbytes & 3) != 0 && lane == 0)
+    *reinterpret_cast<uint16_t*>(b + nbytes - 2) = *reinterpret_cast<const uint16_t*>(src + nbytes - 2);
+  __syncwarp();
+  if (lane < ng) {
+    const uint8_t* gb = b + 26 * lane;
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 26; ++i) {
+      const uint32_t v = gb[i];
+      uint32_t code;
+      if (i < 25) {
+        code = lut[v];
+      } else {
+        // k = 125..127 in digits 0-2; digits 3 and 4 must be the padding value 1
+        code = (v >= 108u && v < 135u) ? (lut[v] & 0x3Fu) : 0x15u;
+      }
+      const int pos = 10 * i;
+      w[pos >> 5] |= code << (pos & 31);
+      if (i < 25 && (pos & 31) > 22) w[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
+    }
+    out[2 * (g0 + lane)] = make_uint4(w[0], w[1], w[2], w[3]);
+    out[2 * (g0 + lane) + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
 }
 
 }  // namespace tb

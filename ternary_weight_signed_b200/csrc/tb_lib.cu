@@ -200,10 +200,13 @@ struct LinearArgs {
   cudaStream_t st;
 };
 
-// Base-3 prefill (more than 16 tokens) re-encodes the weights to 2-bit slots
-// in the workspace, in front of the GEMM's own activations.
+// Base-3 with 8 or more tokens re-encodes the weights to 2-bit slots in the
+// workspace, in front of the activations of the 2-bit path that follows (the
+// tensor-core decode up to 16 tokens, the GEMM beyond): one pass over the
+// base-3 bytes beats a base-3 decode pass per chunk of 4 tokens.
+constexpr int kB3TranscodeMinM = 8;
 size_t b3_transcode_bytes(int f, int64_t M, int64_t N, int64_t K) {
-  if (f != TB_FMT_BASE3 || M <= 16) return 0;
+  if (f != TB_FMT_BASE3 || M < kB3TranscodeMinM) return 0;
   return (static_cast<size_t>(N) * static_cast<size_t>(K / 4) + 255) & ~static_cast<size_t>(255);
 }
 
@@ -449,7 +452,7 @@ constexpr int kB200Sms = 148;
 constexpr int kB200SmemOptin = 232448;
 
 // Base-3 decode serves up to kB3MaxM tokens, in chunks of kGemvMaxM.
-constexpr int kB3MaxM = 16;
+constexpr int kB3MaxM = kB3TranscodeMinM - 1;
 
 bool gemv_ok(const LinearArgs& a) {
   const int64_t maxm = a.f == TB_FMT_BASE3 ? kB3MaxM : kGemvMaxM;
@@ -470,7 +473,9 @@ bool gemv_ok(const LinearArgs& a) {
 
 bool gemv_tc_ok(const LinearArgs& a) {
   GtcPlan pl;
-  return is_float_dtype(a.xt) && a.f == TB_FMT_2BIT && a.M >= 1 && a.M <= kGtcMaxM &&
+  // base-3: after re-encoding to 2-bit slots (8 tokens and more)
+  const bool fmt_ok = a.f == TB_FMT_2BIT || (a.f == TB_FMT_BASE3 && a.M >= kB3TranscodeMinM);
+  return is_float_dtype(a.xt) && fmt_ok && a.M >= 1 && a.M <= kGtcMaxM &&
          a.K % 1024 == 0 && fast_aligned(a) && a.N < (int64_t(1) << 30) &&
          gtc_plan(a.M, a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
 }
@@ -488,8 +493,8 @@ int auto_path(const LinearArgs& a) {
   // does; measured on B200 (K=17408, N=5120) the tensor-core kernel wins from
   // 4 tokens on (31 us against 40 us).
   if (a.f == TB_FMT_2BIT && a.M >= 4 && gemv_tc_ok(a)) return TB_PATH_GEMV_TC;
-  if (gemv_ok(a)) return TB_PATH_GEMV;       // M <= 4 (2-bit), M <= 16 (base-3)
-  if (gemv_tc_ok(a)) return TB_PATH_GEMV_TC;  // 2-bit, up to 16 tokens
+  if (gemv_ok(a)) return TB_PATH_GEMV;       // M <= 4 (2-bit), M <= 7 (base-3)
+  if (gemv_tc_ok(a)) return TB_PATH_GEMV_TC;  // up to 16 tokens (base-3 re-encoded)
   if (gemm_ok(a)) return TB_PATH_GEMM;
   return TB_PATH_SIMPLE;
 }
@@ -672,6 +677,19 @@ tb_status run_gemv_tc_typed(const LinearArgs& a, const DevInfo* d, const GtcPlan
 }
 
 tb_status run_gemv_tc(const LinearArgs& a, const DevInfo* d) {
+  if (a.f == TB_FMT_BASE3) {
+    const size_t tb = b3_transcode_bytes(a.f, a.M, a.N, a.K);
+    const int64_t ngroups = a.N * (a.K / 128);
+    transcode_b3_to_2bit_kernel<<<static_cast<unsigned>((ngroups + 255) / 256), 256, 0, a.st>>>(
+        a.packed, static_cast<uint4*>(a.ws), ngroups);
+    if (launch_status() != TB_OK) return TB_ERR_CUDA;
+    LinearArgs c = a;
+    c.f = TB_FMT_2BIT;
+    c.packed = static_cast<const uint8_t*>(a.ws);
+    c.ws = static_cast<uint8_t*>(a.ws) + tb;
+    c.ws_bytes = a.ws_bytes - tb;
+    return run_gemv_tc(c, d);
+  }
   GtcPlan pl;
   if (!gtc_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
   switch (a.xt) {
@@ -823,7 +841,7 @@ tb_status run_gemm(const LinearArgs& a, const DevInfo* d) {
   const size_t tb = b3_transcode_bytes(a.f, a.M, a.N, a.K);
   const int64_t ngroups = a.N * (a.K / 128);
   transcode_b3_to_2bit_kernel<<<static_cast<unsigned>((ngroups + 255) / 256), 256, 0, a.st>>>(
-      reinterpret_cast<const uint16_t*>(a.packed), static_cast<uint4*>(a.ws), ngroups);
+      a.packed, static_cast<uint4*>(a.ws), ngroups);
   if (launch_status() != TB_OK) return TB_ERR_CUDA;
   LinearArgs c = a;
   c.f = TB_FMT_2BIT;

@@ -124,7 +124,10 @@ def test_path_selection(lib):
     assert p(tb.TB_BF16, "2bit", 16, 5120, 17408) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "2bit", 17, 5120, 17408) == tb.TB_PATH_GEMM
     assert p(tb.TB_BF16, "base3", 1, 17408, 5120) == tb.TB_PATH_GEMV
-    assert p(tb.TB_BF16, "base3", 16, 5120, 17408) == tb.TB_PATH_GEMV
+    assert p(tb.TB_BF16, "base3", 7, 5120, 17408) == tb.TB_PATH_GEMV
+    # 8-16 tokens: re-encoded to 2-bit slots, then the tensor-core decode
+    assert p(tb.TB_BF16, "base3", 8, 5120, 17408) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "base3", 16, 5120, 17408) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "base3", 17, 5120, 17408) == tb.TB_PATH_GEMM
     assert p(tb.TB_BF16, "base3", 2048, 17408, 5120) == tb.TB_PATH_GEMM
     assert p(tb.TB_BF16, "2bit", 1, 256, 1000) == -1

@@ -296,11 +296,20 @@ def test_gemv_tensor_core_more_tokens(m):
     _check(prob.linear(GEMV_TC), ref, prob.p)
 
 
-@pytest.mark.parametrize("m", [5, 16])
+@pytest.mark.parametrize("m", [5, 7])
 def test_gemv_base3_token_chunks(m):
-    """More than four tokens on base-3: one pass over the weights per chunk."""
+    """Five to seven tokens on base-3: one pass over the weights per chunk of four."""
     prob, ref = _problem(26, m, 1001, 2048, 0.33, "base3")
     _check(prob.linear(GEMV), ref, prob.p)
+
+
+@pytest.mark.parametrize("m", [8, 16])
+def test_base3_reencoded_tensor_core_decode(m):
+    """Eight to sixteen tokens on base-3: the weights are re-encoded to 2-bit
+    slots in the workspace, then the tensor-core decode runs on them."""
+    prob, ref = _problem(26, m, 1001, 2048, 0.33, "base3")
+    _check(prob.linear(tb.TB_PATH_GEMV_TC), ref, prob.p)
+    _check(prob.linear(AUTO), ref, prob.p)
 
 
 def test_gemv_tensor_core_rejects_rows_beyond_tmem():
