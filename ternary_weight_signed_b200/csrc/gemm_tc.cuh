@@ -8,10 +8,11 @@
 //   B = fp16(s * t), which is exact because t is -1, 0 or +1 and s is an fp16
 //       value, so no per-group rescaling of the accumulator is needed.
 //
-// Tile: 256 tokens x BN weight rows (BN = 128, 192 or 256, chosen per shape
-// so that the tiles fill whole waves of SMs), K in stages of 64 (one 128-byte
-// swizzle atom of fp16).  The 256 tokens are two M=128 MMAs that share the
-// unpacked B tile, each with its own 128 x BN fp32 accumulator in TMEM.
+// Tile: BM tokens x BN weight rows (BM = 256 or 128; BN = 128, 192 or 256,
+// chosen per shape), K in stages of 64 (one 128-byte swizzle atom of fp16).
+// With BM = 256 the tokens are two M=128 MMAs that share the unpacked B tile,
+// each with its own 128 x BN fp32 accumulator in TMEM; BM = 128 (few tokens)
+// is one MMA and one accumulator.
 // Warp roles:
 //   warp 0    : TMA producer (x' tile with 128B swizzle, packed 2-bit codes);
 //   warp 1    : TMEM allocation and the single thread issuing tcgen05.mma;
@@ -38,23 +39,32 @@
 
 namespace tb {
 
-constexpr int kGemmBM = 256;      // tokens per tile: two MMAs of M = 128
+constexpr int kGemmBM = 256;      // tokens per tile at most: two MMAs of M = 128
 constexpr int kGemmUM = 128;      // M of one MMA (TMEM lanes)
 constexpr int kGemmBN = 256;     // widest weight tile
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 3;
+constexpr int kGemmSmemCap = 227 * 1024;  // dynamic shared memory of one CTA at most
 constexpr int kGemmUnpackWarps = 8;
 constexpr int kGemmThreads = 32 * (2 + kGemmUnpackWarps);
 constexpr int kGemmTmemCols = 512;
-constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 32 KB
-// per weight-tile width BN: B (fp16 s*t) and the packed codes of a stage
+// per tile (BM tokens, BN weight rows): A (fp16 x'), B (fp16 s*t) and the
+// packed codes of a stage
+__host__ __device__ constexpr int gemm_a_bytes(int bm) { return bm * kGemmBK * 2; }
 __host__ __device__ constexpr int gemm_b_bytes(int bn) { return bn * kGemmBK * 2; }
 __host__ __device__ constexpr int gemm_w_bytes(int bn) { return bn * kGemmBK / 4; }
-__host__ __device__ constexpr int gemm_stage_bytes(int bn) { return kGemmABytes + gemm_b_bytes(bn) + gemm_w_bytes(bn); }
-__host__ __device__ constexpr int gemm_smem_bytes(int bn) {
-  return kGemmStages * gemm_stage_bytes(bn) + 1024 /*align*/ + 256 /*barriers*/;
+__host__ __device__ constexpr int gemm_stage_bytes(int bm, int bn) {
+  return gemm_a_bytes(bm) + gemm_b_bytes(bn) + gemm_w_bytes(bn);
 }
-constexpr int kGemmSmemBytes = gemm_smem_bytes(kGemmBN);
+// As many stages as fit (at most 8): small tiles have little MMA work per
+// stage, so more stages are in flight to cover the copies' latency.
+__host__ __device__ constexpr int gemm_stages(int bm, int bn) {
+  return (kGemmSmemCap - 1024 - 256) / gemm_stage_bytes(bm, bn) < 8
+             ? (kGemmSmemCap - 1024 - 256) / gemm_stage_bytes(bm, bn)
+             : 8;
+}
+__host__ __device__ constexpr int gemm_smem_bytes(int bm, int bn) {
+  return gemm_stages(bm, bn) * gemm_stage_bytes(bm, bn) + 1024 /*align*/ + 256 /*barriers*/;
+}
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B fp16
 // (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
@@ -197,12 +207,15 @@ __device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, c
   }
 }
 
-template <int BN, typename TOut>
+template <int BM, int BN, typename TOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_2bit_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                         const GemmParams p) {
   static_assert(BN % 32 == 0 && BN >= 128 && BN <= kGemmBN, "weight tile width");
-  constexpr int kStage = gemm_stage_bytes(BN), kB = gemm_b_bytes(BN), kW = gemm_w_bytes(BN);
+  static_assert(BM == 128 || BM == 256, "token tile");
+  constexpr int kA = gemm_a_bytes(BM), kStage = gemm_stage_bytes(BM, BN), kB = gemm_b_bytes(BN),
+                kW = gemm_w_bytes(BN), kGemmStages = gemm_stages(BM, BN);
+  static_assert(kGemmStages >= 2, "two stages at least");
   constexpr uint32_t kIdesc = gemm_idesc(BN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -213,7 +226,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kGemmBM;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
   const int nk = p.K / kGemmBK;
 
   if (threadIdx.x == 0) {
@@ -246,9 +259,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             !mbar_wait(&empty[s], ((kb / kGemmStages) & 1) ^ 1, FAULT_WAIT_EMPTY))
           break;
         uint8_t* st = smem + s * kStage;
-        mbar_arrive_expect_tx(&full[s], kGemmABytes + kW);
+        mbar_arrive_expect_tx(&full[s], kA + kW);
         tma_load_2d(st, &tm_x, kb * kGemmBK, m0, &full[s]);
-        tma_load_2d(st + kGemmABytes + kB, &tm_w, kb * (kGemmBK / 16), n0, &full[s]);
+        tma_load_2d(st + kA + kB, &tm_w, kb * (kGemmBK / 16), n0, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -262,13 +275,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t a = smem_u32(smem + s * kStage);
-        const uint32_t b = a + kGemmABytes;
+        const uint32_t b = a + kA;
 #pragma unroll
         for (int kk = 0; kk < kGemmBK / 16; ++kk) {
           const uint64_t bd = umma_desc_sw128(b + 32 * kk);
           const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
           umma_f16(tmem, umma_desc_sw128(a + 32 * kk), bd, kIdesc, acc);
-          umma_f16(tmem + BN, umma_desc_sw128(a + kGemmUM * 128 + 32 * kk), bd, kIdesc, acc);
+          if constexpr (BM == 256)
+            umma_f16(tmem + BN, umma_desc_sw128(a + kGemmUM * 128 + 32 * kk), bd, kIdesc, acc);
         }
         umma_commit(&empty[s]);
       }
@@ -302,10 +316,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (g + 1 < G) s_next = __ushort_as_half(row_ok ? srow[g + 1] : uint16_t(0));
       }
       uint8_t* st = smem + s * kStage;
-      const uint4 w4 = in_tile ? *reinterpret_cast<const uint4*>(st + kGemmABytes + kB + r * 16) : make_uint4(0, 0, 0, 0);
+      const uint4 w4 = in_tile ? *reinterpret_cast<const uint4*>(st + kA + kB + r * 16) : make_uint4(0, 0, 0, 0);
       const __half2 s2 = __halves2half2(s_cur, s_cur);
       const __half2 ns2 = __hneg2(s2);
-      uint8_t* row = st + kGemmABytes + r * 128;
+      uint8_t* row = st + kA + r * 128;
 #pragma unroll
       for (int wd = 0; wd < 4 && in_tile; ++wd) {
         const uint32_t w = (&w4.x)[wd];
@@ -333,14 +347,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (mbar_wait(accum, 0, FAULT_WAIT_EPILOGUE)) {
       tc_fence_after();
       const int q = warp & 3;             // TMEM lane quarter this warp may access
-      const int h = (warp - 2) >> 2;      // which of the two accumulators
-      const int m = m0 + kGemmUM * h + 32 * q + lane;
+      const int h = (warp - 2) >> 2;      // BM = 256: which accumulator; BM = 128: which half of the columns
+      const int m = m0 + (BM == 256 ? kGemmUM * h : 0) + 32 * q + lane;
       TOut* y = reinterpret_cast<TOut*>(p.y);
       const bool vec = (p.N % static_cast<int>(16 / sizeof(TOut))) == 0;  // 16-byte row alignment
+      constexpr int kCols = BM == 256 ? BN / 32 : BN / 64;  // 32-column chunks per warp
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int cc = 0; cc < kCols; ++cc) {
+        const int c = BM == 256 ? cc : h * kCols + cc;
         uint32_t v32[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(BN * h + 32 * c), v32);
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) +
+                      static_cast<uint32_t>((BM == 256 ? BN * h : 0) + 32 * c),
+                  v32);
         tmem_ld_wait();
         const int nb = n0 + 32 * c;
         if (m < p.M && nb < p.N) {

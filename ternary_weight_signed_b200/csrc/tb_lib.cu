@@ -484,7 +484,7 @@ bool gemm_ok(const LinearArgs& a) {
   // base-3 is served by re-encoding to 2-bit slots first (more than 16 tokens)
   if (a.f == TB_FMT_BASE3 && a.M <= 16) return false;
   return is_float_dtype(a.xt) && a.K % 1024 == 0 && fast_aligned(a) &&
-         (a.M + kGemmBM - 1) / kGemmBM <= 65535 && a.N < (int64_t(1) << 30);
+         (a.M + kGemmUM - 1) / kGemmUM <= 65535 && a.N < (int64_t(1) << 30);
 }
 
 int auto_path(const LinearArgs& a) {
@@ -859,12 +859,16 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
     default: launch_prep_gemm<float>(a, xh); break;
   }
   if (launch_status() != TB_OK) return TB_ERR_CUDA;
+  // Token tile: 128 when it pads fewer token rows than 256 (up to 128 tokens,
+  // and e.g. 300 tokens: 384 against 512 rows), else 256, whose two MMAs share
+  // each unpacked weight tile.
+  const int bm = ((a.M + 127) / 128) * 128 < ((a.M + 255) / 256) * 256 ? 128 : 256;
   // Weight-tile width: wave fill of the SMs times the tile's own efficiency.
   // Narrower tiles reuse each activation stage for fewer weight rows and leave
   // unpack warps idle; on B200 the 192-wide tile ran the prefill shape
   // (2048 x 17408 x 5120) at 0.90 of the 256-wide tile's per-tile rate, which
   // its better wave fill (4.92 against 3.68 waves) does not make up.
-  const int64_t mt = (a.M + kGemmBM - 1) / kGemmBM;
+  const int64_t mt = (a.M + bm - 1) / bm;
   int bn = 256;
   double best = -1.0;
   const int cands[3] = {256, 192, 128};
@@ -879,8 +883,8 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
     }
   }
   CUtensorMap tm_x, tm_w;
-  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGemmBK, kGemmBM,
-                  CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGemmBK,
+                  static_cast<uint32_t>(bm), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
   if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, kGemmBK / 16,
                   static_cast<uint32_t>(bn)) != TB_OK)
@@ -892,20 +896,25 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   gp.y = a.y;
   gp.scales = a.scales;
   const dim3 grid(static_cast<unsigned>((a.N + bn - 1) / bn), static_cast<unsigned>(mt));
-#define TB_GEMM_LAUNCH(BN)                                                                                   \
-  if (bn == BN) {                                                                                            \
-    if (a.yt == TB_FP32) {                                                                                   \
-      auto k = gemm_2bit_tc_kernel<BN, float>;                                                               \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
-      return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BN)), a.st, tm_x, tm_w, gp); \
-    }                                                                                                        \
-    auto k = gemm_2bit_tc_kernel<BN, __nv_bfloat16>;                                                         \
-    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                       \
-    return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BN)), a.st, tm_x, tm_w, gp);   \
+#define TB_GEMM_LAUNCH(BM, BN)                                                                             \
+  if (bm == BM && bn == BN) {                                                                              \
+    if (a.yt == TB_FP32) {                                                                                 \
+      auto k = gemm_2bit_tc_kernel<BM, BN, float>;                                                         \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                   \
+      return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BM, BN)), a.st, tm_x, \
+                        tm_w, gp);                                                                         \
+    }                                                                                                      \
+    auto k = gemm_2bit_tc_kernel<BM, BN, __nv_bfloat16>;                                                   \
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
+    return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BM, BN)), a.st, tm_x,   \
+                      tm_w, gp);                                                                           \
   }
-  TB_GEMM_LAUNCH(256)
-  TB_GEMM_LAUNCH(192)
-  TB_GEMM_LAUNCH(128)
+  TB_GEMM_LAUNCH(256, 256)
+  TB_GEMM_LAUNCH(256, 192)
+  TB_GEMM_LAUNCH(256, 128)
+  TB_GEMM_LAUNCH(128, 256)
+  TB_GEMM_LAUNCH(128, 192)
+  TB_GEMM_LAUNCH(128, 128)
 #undef TB_GEMM_LAUNCH
   return TB_ERR_SHAPE;
 }
