@@ -175,9 +175,11 @@ tb_status tb_ternary_linear(const void* x, tb_dtype xt, const uint8_t* packed,
 
 /* tb_ternary_linear with the kernel path chosen by the caller (tests, tuning).
  * A path that cannot take the arguments returns TB_ERR_SHAPE without launching
- * anything: GEMV needs float mode, M <= 4, K % 1024 == 0 and 16-byte aligned
- * packed/scales; GEMM needs float mode, K % 1024 == 0 and aligned pointers;
- * SIMPLE takes everything tb_ternary_linear takes. */
+ * anything: GEMV needs float mode, M <= 4 (base-3: M <= 7), K % 1024 == 0 and
+ * 16-byte aligned packed/scales; GEMV_TC needs float mode, M <= 16 (base-3:
+ * 8 <= M <= 16), K % 1024 == 0, aligned pointers and a plan that fits the
+ * SMs; GEMM needs float mode, K % 1024 == 0 and aligned pointers (base-3:
+ * M > 16); SIMPLE takes everything tb_ternary_linear takes. */
 tb_status tb_ternary_linear_ex(const void* x, tb_dtype xt, const uint8_t* packed,
                                const uint16_t* scales, tb_format f, int64_t M, int64_t N,
                                int64_t K, const int8_t* signs, void* y, tb_dtype yt,
