@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   const int G = p.K / 128;
   const int r0 = blockIdx.x * p.R;
   const int nrows = min(p.R, p.N - r0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const uint32_t wbytes = static_cast<uint32_t>(p.NB) * static_cast<uint32_t>(p.R) * 128u;
   const uint32_t abytes = static_cast<uint32_t>(gemv_act_stage_bytes(1, p.NB));
   const int act_off = p.NB * p.box_stride;

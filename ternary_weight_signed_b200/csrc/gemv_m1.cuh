@@ -21,9 +21,10 @@
 //
 // Rotation (news.ditty.ir, second and third paragraphs; openbonsai.org, "How
 // it works", "Rotate"): x'_b = H (d_b * x_b) / 32 on each 1024-block, H the
-// Sylvester matrix.  One warp rotates one block: lane a holds elements
-// 32 a .. 32 a + 31; the transform over the low five index bits runs inside
-// the lane, over the high five bits across lanes (butterflies by shuffle), so
+// Sylvester matrix.  One warp rotates one block: lane c first holds elements
+// 32 r + c (r = 0..31) and transforms over the high five index bits inside
+// the lane; a transpose through shared memory gives lane a the elements
+// 32 a .. 32 a + 31, transformed over the low five bits inside the lane, so
 // lane a ends with x'[32 a .. 32 a + 31], a quarter of group a / 4.  The 1/32
 // is exact and is folded into the fixed-point scale.
 //
@@ -69,6 +70,12 @@ constexpr int kG1MaxRows = 256;  // TMA box height limit
 // longer K goes through prep_gemv1_kernel.
 constexpr int kG1FusedMaxBlocks = kG1Warps;
 constexpr int kG1GroupBytes = 256;
+// Groups sit 272 bytes apart in shared memory: the four groups of a chunk,
+// read together by the four quarter-warps, then start in four different
+// 16-byte bank groups and one load serves all four in a single pass.
+constexpr int kG1GroupStride = kG1GroupBytes + 16;
+// A block's 8 groups of words double as its warp's 2 KB transpose buffer.
+static_assert(8 * kG1GroupStride >= 512 * 4, "transpose buffer");
 
 // d = c + a.lo16 * b.byte0 + a.hi16 * b.byte1 (lo) or * bytes 2, 3 (hi);
 // a signed 16-bit, b unsigned 8-bit.
@@ -102,7 +109,8 @@ struct Gemv1Params {
 
 // Shared memory (offsets from the 1 KB-aligned base; 1 KB of slack in front):
 //   ring  nslots x slot_bytes
-//   act   G x 256 bytes of activation words, then G x {float e_g, int sum q}
+//   act   G x 272 bytes (256 of activation words, 16 of padding), then G x
+//         {float e_g, int sum q}
 //   sc    R x G fp16 scales of the CTA's rows
 //   red   Wk x R fp32 row sums of the warps (before that, the exchange
 //         buffer of the two-warp rotation: 4 KB per 1024-block)
@@ -111,7 +119,7 @@ struct Gemv1Layout {
   int off_act, off_sc, off_red, off_bar;
   int64_t bytes;
 };
-__host__ __device__ inline int64_t g1_act_bytes(int64_t K) { return (K / 128) * (kG1GroupBytes + 8); }
+__host__ __device__ inline int64_t g1_act_bytes(int64_t K) { return (K / 128) * (kG1GroupStride + 8); }
 // Two warps rotate each 1024-block when there are warps enough for that.
 __host__ __device__ constexpr bool g1_half_blocks(int64_t K) { return 2 * (K / 1024) <= kG1Warps; }
 __host__ __device__ inline Gemv1Layout gemv1_layout(int64_t K, int R, int Wk, int nstage, int64_t ring_bytes) {
@@ -128,57 +136,86 @@ __host__ __device__ inline Gemv1Layout gemv1_layout(int64_t K, int R, int Wk, in
 }
 
 // ---------------------------------------------------------------- rotation
-// The lane's 32 signs of block `blk` as packed bytes (loaded before the wait
-// for the previous kernel: signs are parameters of the layer).
-__device__ __forceinline__ void g1_load_signs(const int8_t* signs, int blk, int lane, uint32_t (&sg)[8]) {
-  const uint4* p = reinterpret_cast<const uint4*>(signs + static_cast<int64_t>(blk) * kHB + 32 * lane);
-  const uint4 a = p[0], b = p[1];
-  sg[0] = a.x; sg[1] = a.y; sg[2] = a.z; sg[3] = a.w;
-  sg[4] = b.x; sg[5] = b.y; sg[6] = b.z; sg[7] = b.w;
-}
-
 template <typename T>
 __device__ __forceinline__ void g1_load32(const T* p, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) load8<T>(p + 8 * i, v + 8 * i);
 }
 
-// One warp: rotate 1024-block `blk` (with signs `sg` when has_signs, else
-// x is taken as already rotated) and write its 8 groups' activation words and
-// info into `act` (G groups of words, then G infos).
-template <typename TIn>
-__device__ __forceinline__ void g1_rotate_block(const TIn* __restrict__ x, const uint32_t (&sg)[8], bool has_signs,
-                                                int blk, int G, uint8_t* act, int lane) {
-  float v[32];
-  g1_load32<TIn>(x + static_cast<int64_t>(blk) * kHB + 32 * lane, v);
-  float scale = 1.f;
-  if (has_signs) {
-    // sign byte 0xFF (-1) flips the float's sign bit
+// Radix-2 butterflies over the five index bits held in the lane (v[i], i the
+// bits): after it v holds the 32-point Sylvester transform of the input.
+__device__ __forceinline__ void g1_fwht32(float (&v)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const uint32_t sbit = (sg[i >> 2] << (24 - 8 * (i & 3))) & 0x80000000u;
-      v[i] = __int_as_float(__float_as_int(v[i]) ^ static_cast<int>(sbit));
-    }
-    // low five index bits: inside the lane
-#pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if ((i & h) == 0) {
-          const float a = v[i], b = v[i + h];
-          v[i] = a + b;
-          v[i + h] = a - b;
-        }
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
       }
     }
-    // high five index bits: across lanes (lower partner keeps a + b, upper gets a - b)
+  }
+}
+
+// One warp: rotate 1024-block `blk` (with the block's 1024 signs `sgn`, in
+// shared or global memory, when not null; else x is taken as already rotated)
+// and write its 8 groups' activation words and info into `act` (G groups of
+// words, then G infos).  When `sbar` is not null the signs arrive by a bulk
+// copy completing on it.  `xbuf` is 2 KB of shared memory of this warp's own
+// (16 rows of 32 floats); it may overlap the signs.  False if the wait for
+// the signs gave up.
+//
+// With index k = 32 r + c, H_1024 = H_32 (x) H_32: lane c loads x[32 r + c]
+// for r = 0..31 (each load instruction reads 32 consecutive elements) and
+// transforms over r inside the lane; the 32 x 32 tile is transposed through
+// xbuf (two halves of 16 rows; the 16-byte column chunks XOR-swizzled by the
+// row, so neither the 4-byte stores of a row nor the 16-byte loads of a
+// quarter-warp meet a bank twice); lane r then holds the 32 values of row r
+// and transforms over c.  Lane a ends with x'[32 a .. 32 a + 31].
+template <typename TIn>
+__device__ __forceinline__ bool g1_rotate_block(const TIn* __restrict__ x, const int8_t* sgn, uint64_t* sbar,
+                                                int blk, int G, uint8_t* act, float* xbuf, int lane) {
+  const TIn* xb = x + static_cast<int64_t>(blk) * kHB;
+  float v[32];
+  float scale = 1.f;
+  if (sgn != nullptr) {
 #pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-      const float sgn = (lane & m) ? -1.f : 1.f;
+    for (int i = 0; i < 32; ++i) v[i] = to_f32<TIn>(xb[32 * i + lane]);
+    // signs staged in shared memory by a bulk copy: wait for it while the
+    // loads of x are in flight
+    if (sbar != nullptr && !__all_sync(0xffffffffu, mbar_wait(sbar, 0, FAULT_WAIT_ACT))) return false;
+    // sign byte -1 (0xFF) flips the float's sign bit
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fmaf(sgn, v[i], __shfl_xor_sync(0xffffffffu, v[i], m));
+    for (int i = 0; i < 32; ++i)
+      v[i] = __int_as_float(__float_as_int(v[i]) ^ (static_cast<int32_t>(sgn[32 * i + lane]) & INT32_MIN));
+    __syncwarp();  // the signs may share memory with xbuf
+    g1_fwht32(v);
+    float u[32];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) xbuf[32 * r + ((((lane >> 2) ^ r) & 7) << 2) + (lane & 3)] = v[16 * hf + r];
+      __syncwarp();
+      if ((lane >> 4) == hf) {
+        const float4* row = reinterpret_cast<const float4*>(xbuf + 32 * (lane & 15));
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 t = row[q ^ (lane & 7)];
+          u[4 * q] = t.x;
+          u[4 * q + 1] = t.y;
+          u[4 * q + 2] = t.z;
+          u[4 * q + 3] = t.w;
+        }
+      }
+      __syncwarp();
     }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = u[i];
+    g1_fwht32(v);
     scale = kHNorm;
+  } else {
+    g1_load32<TIn>(xb + 32 * lane, v);
   }
   // 16-bit fixed point of the group (4 lanes): e = max|x'| / kQMax with x' = scale * v
   float mx = 0.f;
@@ -188,15 +225,20 @@ __device__ __forceinline__ void g1_rotate_block(const TIn* __restrict__ x, const
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   mx *= scale;  // exact (a power of two)
   const float e = mx / kQMax;
-  // inv * scale is exact too, so q = rint(x' * kQMax / max|x'|) as in prep_gemv_kernel
+  // inv * scale is exact too, so q = rint(x' * kQMax / max|x'|) as in
+  // prep_gemv_kernel.  The rounding adds 1.5 * 2^23: for |f| <= kQMax the sum's
+  // bits are 0x4B400000 + rint(f) (round to nearest even), so their low 16
+  // bits are q as int16.
   const float inv = mx > 0.f ? (kQMax / mx) * scale : 0.f;
-  int q[32];
-  int qs = 0;
+  uint32_t qb[32];
+  uint32_t qsb = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    q[i] = max(-32512, min(32512, __float2int_rn(v[i] * inv)));
-    qs += q[i];
+    const float f = fminf(fmaxf(__fmul_rn(v[i], inv), -kQMax), kQMax);
+    qb[i] = __float_as_uint(__fadd_rn(f, 12582912.0f));
+    qsb += qb[i];
   }
+  int qs = static_cast<int>(qsb - 32u * 0x4B400000u);
   qs += __shfl_xor_sync(0xffffffffu, qs, 1);
   qs += __shfl_xor_sync(0xffffffffu, qs, 2);
   // lane a holds codes 32 (a & 3) .. + 31 of group a >> 2, i.e. words
@@ -210,18 +252,19 @@ __device__ __forceinline__ void g1_rotate_block(const TIn* __restrict__ x, const
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int u = 16 * i2 + 8 * h + j;
-        wv[8 * i2 + 2 * j + h] = __byte_perm(static_cast<uint32_t>(q[u]), static_cast<uint32_t>(q[u + 4]), 0x5410);
+        wv[8 * i2 + 2 * j + h] = __byte_perm(qb[u], qb[u + 4], 0x5410);
       }
   const int g = blk * 8 + (lane >> 2);
-  uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupBytes + 64 * (lane & 3));
+  uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupStride + 64 * (lane & 3));
 #pragma unroll
   for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
   if ((lane & 3) == 0) {
     int2 inf;
     inf.x = __float_as_int(e);
     inf.y = qs;
-    reinterpret_cast<int2*>(act + G * kG1GroupBytes)[g] = inf;
+    reinterpret_cast<int2*>(act + G * kG1GroupStride)[g] = inf;
   }
+  return true;
 }
 
 // Two warps, halves hf = 0, 1 of 1024-block `blk`: lane l of half hf holds
@@ -303,14 +346,14 @@ __device__ __forceinline__ void g1_rotate_half(const TIn* __restrict__ x, const 
     for (int h = 0; h < 2; ++h)
       wv[2 * j + h] = __byte_perm(static_cast<uint32_t>(q[8 * h + j]), static_cast<uint32_t>(q[8 * h + j + 4]), 0x5410);
   const int g = blk * 8 + 4 * hf + (lane >> 3);
-  uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupBytes + 32 * (lane & 7));
+  uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupStride + 32 * (lane & 7));
   dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
   dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
   if ((lane & 7) == 0) {
     int2 inf;
     inf.x = __float_as_int(e);
     inf.y = qs;
-    reinterpret_cast<int2*>(act + G * kG1GroupBytes)[g] = inf;
+    reinterpret_cast<int2*>(act + G * kG1GroupStride)[g] = inf;
   }
 }
 
@@ -321,14 +364,15 @@ __device__ __forceinline__ void g1_rotate_half(const TIn* __restrict__ x, const 
 template <typename TIn>
 __global__ void __launch_bounds__(128) prep_gemv1_kernel(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
                                                          uint8_t* __restrict__ ws, int K) {
+  __shared__ __align__(16) float xbuf[4][512];
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int blk = blockIdx.x * 4 + (threadIdx.x >> 5);
   const bool live = blk < (K >> 10);
-  uint32_t sg[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  if (live && signs != nullptr) g1_load_signs(signs, blk, lane, sg);
   pdl_wait();
-  if (live) g1_rotate_block<TIn>(x, sg, signs != nullptr, blk, K >> 7, ws, lane);
+  if (live)
+    g1_rotate_block<TIn>(x, signs != nullptr ? signs + static_cast<int64_t>(blk) * kHB : nullptr, nullptr, blk,
+                         K >> 7, ws, xbuf[threadIdx.x >> 5], lane);
 }
 
 // ---------------------------------------------------------------- decode
@@ -406,8 +450,15 @@ __global__ void __launch_bounds__(kG1Threads, 2)
     if (warp == kG1Warps - 1) {
       const uint32_t sbytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(G * 2);
       const uint32_t abytes = kFused ? 0u : static_cast<uint32_t>(g1_act_bytes(p.K));
-      mbar_arrive_expect_tx(pre_bar, sbytes + abytes);
+      // one warp per block: the block's signs go to the start of its slice of
+      // the activation words
+      const bool stage_signs = kFused && p.signs != nullptr && !g1_half_blocks(p.K);
+      const uint32_t gbytes = stage_signs ? static_cast<uint32_t>(p.K) : 0u;
+      mbar_arrive_expect_tx(pre_bar, sbytes + abytes + gbytes);
       bulk_load(base + p.off_sc, p.scales + static_cast<int64_t>(r0) * G, sbytes, pre_bar);
+      if (stage_signs)
+        for (int b = 0; b < (p.K >> 10); ++b)
+          bulk_load(act + b * 8 * kG1GroupStride, p.signs + static_cast<int64_t>(b) * kHB, kHB, pre_bar);
     }
     for (int s = kG1Warps - 1 - warp; s < pre; s += kG1Warps) gemv1_issue(&tm_w, p, ring, &full[s], s, s, r0);
     if constexpr (!kFused) {
@@ -425,13 +476,17 @@ __global__ void __launch_bounds__(kG1Threads, 2)
       if (warp < 2 * nblk)
         g1_rotate_half<TIn>(x, p.signs, warp >> 1, warp & 1, G, act, red + (warp >> 1) * kHB, 1 + (warp >> 1), lane);
     } else {
-      // block `warp` (K <= kG1FusedMaxBlocks blocks); its signs are loaded
-      // before the wait
-      uint32_t sg[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      // block `warp` (K <= kG1FusedMaxBlocks blocks); its signs were staged
+      // in shared memory before the wait
       const bool live = warp < nblk;
-      if (live && p.signs != nullptr) g1_load_signs(p.signs, warp, lane, sg);
       pdl_wait();  // x may be the previous kernel's output
-      if (live) g1_rotate_block<TIn>(x, sg, p.signs != nullptr, warp, G, act, lane);
+      // the transpose buffer is this block's own slice of the activation words
+      // (8 x 272 bytes, written only after the transpose)
+      uint8_t* slice = act + warp * 8 * kG1GroupStride;
+      if (live && !g1_rotate_block<TIn>(x, p.signs != nullptr ? reinterpret_cast<const int8_t*>(slice) : nullptr,
+                                        pre_bar, warp, G, act, reinterpret_cast<float*>(slice), lane) &&
+          lane == 0)
+        atomicExch(cta_fault, 1u);
     }
   }
   __syncthreads();
@@ -440,7 +495,7 @@ __global__ void __launch_bounds__(kG1Threads, 2)
   const int tg = warp / p.Wk, wk = warp - tg * p.Wk;
   const bool active = tg < p.Wt;
   const int t0 = tg * p.RT / p.Wt, nt = active ? (tg + 1) * p.RT / p.Wt - t0 : 0;  // this warp's row tiles
-  const int2* info = reinterpret_cast<const int2*>(act + G * kG1GroupBytes);
+  const int2* info = reinterpret_cast<const int2*>(act + G * kG1GroupStride);
   // byte offsets in a box of the lane's two 16-byte pieces (2 gslot and
   // 2 gslot + 1 of the row's 128 bytes, swizzled with the row index mod 8 =
   // rsub) and of the rows' scales; rows past the CTA's end read valid rows
@@ -472,7 +527,7 @@ __global__ void __launch_bounds__(kG1Threads, 2)
     const uint8_t* box = sbase + (c - (s << p.nb_log2)) * p.box_stride;
     const int g = 4 * c + gslot;
     uint32_t A[64];
-    const uint4* src = reinterpret_cast<const uint4*>(act + g * kG1GroupBytes);
+    const uint4* src = reinterpret_cast<const uint4*>(act + g * kG1GroupStride);
 #pragma unroll
     for (int v = 0; v < 16; ++v) {
       const uint4 u4 = src[v];

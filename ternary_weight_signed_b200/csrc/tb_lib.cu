@@ -318,7 +318,6 @@ bool g1_plan(int64_t N, int64_t K, int sm_count, int max_smem, bool fused, G1Pla
   }
   if (best_cost < 0) return false;
   pl.box_stride = static_cast<int>(align_up(R * 128, 1024));
-  // stages of at least 8 KB of weights
   // stages of at least 8 KB of weights, a power of two of chunks
   int64_t want = (8192 + R * 128 - 1) / (R * 128);
   if (want > C) want = C;
