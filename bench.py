@@ -37,6 +37,25 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 
 
+def _barrier(world):
+    """All ranks meet here (no-op on one GPU)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x, dev, world):
+    """The largest of the ranks' values of x: a job takes as long as its
+    slowest rank.  x itself on one GPU."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -199,9 +218,7 @@ def measure_decode(args, tb, inputs, dev, stream, fmt, m, n, k, seed, p0, scale_
     sampler = ClockSampler(torch.cuda.current_device()) if sample else None
     if sampler:
         sampler.start()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    _barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -212,14 +229,9 @@ def measure_decode(args, tb, inputs, dev, stream, fmt, m, n, k, seed, p0, scale_
         e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = e0.elapsed_time(e1)
+    _barrier(world)
+    ms = _max_over_ranks(e0.elapsed_time(e1), dev, world)
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     del g_main
     steps = reps * chunk
     return {"ms_per_step": ms / steps, "steps": steps, "step_bytes": step_bytes, "copies": copies,
@@ -283,9 +295,8 @@ def measure_e2e(args, tb, dev, stream, fmt, m, n, k, prob, world):
         g.replay()
     torch.cuda.synchronize()
     reps = max(1, min(args.steps, 20 * chunk) // chunk)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    _barrier(world)
+    torch.cuda.synchronize()
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -294,11 +305,9 @@ def measure_e2e(args, tb, dev, stream, fmt, m, n, k, prob, world):
             g.replay()
         a1.record(stream)
     a1.synchronize()
-    ms = a0.elapsed_time(a1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    torch.cuda.synchronize()
+    _barrier(world)
+    ms = _max_over_ranks(a0.elapsed_time(a1), dev, world)
     del g
     e2e_ms = ms / (reps * chunk)
     step_bytes = _packed_bytes(fmt, n, k)
@@ -349,7 +358,7 @@ def run_ours(args, rank, world):
             others[fmt] = _decode_entry(res, peak, peak_kind, world)
         res.pop("problem")
         torch.cuda.empty_cache()
-    prefill = run_prefill(args, dev, stream, tb, inputs) if args.prefill else None
+    prefill = run_prefill(args, dev, stream, tb, inputs, world) if args.prefill else None
     head = _decode_entry(main, peak, peak_kind, world)
     roof = head["roofline"]
     roof["traffic"] = _traffic(args.fmt)
@@ -367,7 +376,8 @@ def run_ours(args, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "u8 codes, fp16 scales, bf16 x -> fp32 (int8x2 dp4a on 16-bit fixed point, fp32 scale)",
+        "dtype": "u8 codes, fp16 scales, bf16 x -> fp32 (dp2a: u8 codes x int16 fixed-point x', exact int32 per "
+                 "group, fp32 scale)",
         "data": "synthetic (seeded; codes P(0)=0.33, |N(0,1)|*0.02 fp16 scales, N(0,1) bf16 x with 1% +-20 outliers)",
         "config": {"workload": f"decode GEMV gate/up M=1 K=5120 N=17408 ({args.fmt} packing)",
                    "M": m, "K": k, "N": n, "format": args.fmt, "kernel_path": main["path"],
@@ -384,10 +394,12 @@ def run_ours(args, rank, world):
     }
 
 
-def run_prefill(args, dev, stream, tb, inputs):
-    """Prefill GEMM workload (M=2048 tokens, K=5120, N=17408, 2-bit): tokens/s,
-    TFLOP-equivalent/s (2*M*N*K per call) and its fraction of the measured dense
-    16-bit tensor peak.  Two weight copies alternate; the call is compute-bound."""
+def run_prefill(args, dev, stream, tb, inputs, world=1):
+    """Prefill GEMM workload (M=2048 tokens, K=5120, N=17408, 2-bit): tokens/s
+    of the whole job (every rank one replica, timed as the slowest rank),
+    TFLOP-equivalent/s per GPU (2*M*N*K per call) and its fraction of the
+    measured dense 16-bit tensor peak.  Two weight copies alternate; the call
+    is compute-bound."""
     import torch
 
     w = inputs.WORKLOADS["prefill_m2048_k5120_n17408"]
@@ -421,6 +433,8 @@ def run_prefill(args, dev, stream, tb, inputs):
                 call(i)
         g.replay()
     stream.synchronize()
+    _barrier(world)
+    torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -428,12 +442,14 @@ def run_prefill(args, dev, stream, tb, inputs):
         g.replay()
         e1.record(stream)
     e1.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    torch.cuda.synchronize()
+    _barrier(world)
+    ms = _max_over_ranks(e0.elapsed_time(e1), dev, world) / steps
     flops = 2.0 * m * n * k
     tflops = flops / (ms * 1e-3) / 1e12
     peak, kind = _tensor_peak()
     return {"workload": "prefill GEMM M=2048 K=5120 N=17408 (2bit), bf16 in/out",
-            "tok_s": round(m / (ms * 1e-3), 1), "ms_per_call": round(ms, 5), "steps": steps,
+            "tok_s": round(m * world / (ms * 1e-3), 1), "ms_per_call": round(ms, 5), "steps": steps,
             "tflops_equiv": round(tflops, 2),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
