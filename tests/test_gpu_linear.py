@@ -65,6 +65,9 @@ WORKLOAD_CASES = [
     (14, 2, 17408, 5120, 0.33, "abs_normal", 0.01),    # gate/up, two tokens (two-CTA decode kernel)
     (15, 4, 17408, 5120, 0.33, "abs_normal", 0.0),     # gate/up, four tokens
     (16, 3, 9999, 3072, 0.5, "abs_normal", 0.0),       # three tokens in a four-token kernel, ragged N
+    (17, 1, 4000, 8192, 0.33, "abs_normal", 0.01),     # one token, 8 blocks: every warp rotates one
+    (18, 1, 3000, 7168, 0.5, "abs_normal", 0.0),       # one token, 7 blocks, ragged rows per CTA
+    (19, 1, 10000, 9216, 0.33, "abs_normal", 0.0),     # one token, 9 blocks: activation kernel, then decode
 ]
 
 
@@ -124,6 +127,17 @@ def test_other_input_dtypes(path, xt, fmt):
     ref = orc.linear(xv, prob.p.codes, prob.p.scales, prob.p.signs)
     y = prob.linear(path, x=x, xt=xt)
     _check(y, ref, prob.p)
+
+
+@pytest.mark.parametrize("xt", [tb.TB_FP16, tb.TB_FP32])
+def test_one_token_input_dtypes(xt):
+    """fp16 and fp32 activations through the one-token kernel's own rotation
+    (strided loads of x, one warp per 1024-block)."""
+    prob, _ = _problem(23, 1, 2000, 5120, 0.33, "2bit", "abs_normal", 0.01)
+    x = torch.from_numpy(prob.p.x).to(DEV).to(torch.float16 if xt == tb.TB_FP16 else torch.float32)
+    ref = orc.linear(x.double().cpu().numpy(), prob.p.codes, prob.p.scales, prob.p.signs)
+    _check(prob.linear(GEMV, x=x, xt=xt), ref, prob.p)
+    _check(prob.linear(GEMV, x=x, xt=xt, yt=tb.TB_BF16), ref, prob.p)
 
 
 @pytest.mark.parametrize("fmt", ["2bit", "base3"])
