@@ -37,6 +37,12 @@ Readings taken where the pages are silent (each is stated again in the design doc):
   all codes it carries decode to t = 0 and it is counted once.
 * Codes outside {-1, 0, 1} given to the packer are packed as t = 0 and counted.
 * Integer mode: y[m, n] = sum_k t[n, k] x[m, k] for int8 x, no scales, no rotation.
+* Producer side (openbonsai.org, "How it works", steps 1 "Rotate" and 2
+  "Round"): the pages round with sequential GPTQ on calibration data, which
+  needs a model and data; the stand-in here is plain rounding to the nearest
+  level with one scale per group.  The scale is the group's mean |w'| (after
+  the fold), rounded to fp16; t = clip(rint(w' / s), -1, 1) with that fp16 s
+  (rint: halves to even); a group of zeros gets s = 0 and t = 0.
 
 Parity: every function here is pinned by the CPU tests (closed forms,
 exhaustive byte tables, brute force, library routines); none is "parity
@@ -102,9 +108,54 @@ def rotate(x: np.ndarray, signs: np.ndarray, inverse: bool = False) -> np.ndarra
     return out
 
 
+def fold_weights(w: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """W' = W R for a dense W [N, K]: block b of every row times R_b
+    (explicit fp64 products; the run time then applies R^T to x)."""
+    w = np.atleast_2d(np.asarray(w, dtype=np.float64))
+    n, k = w.shape
+    if k % BLOCK:
+        raise ValueError("K must be a multiple of 1024")
+    signs = np.asarray(signs)
+    if signs.shape != (k,):
+        raise ValueError("one sign per input coordinate expected")
+    out = np.empty_like(w)
+    for b in range(k // BLOCK):
+        sl = slice(b * BLOCK, (b + 1) * BLOCK)
+        out[:, sl] = w[:, sl] @ rotation_matrix(signs[sl])
+    return out
+
+
 # --------------------------------------------------------------------------
 # Ternary g128 weights
 # --------------------------------------------------------------------------
+
+def ternarize(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Round a dense [N, K] matrix to ternary g128: per 128-group the scale
+    s = fp16(mean |w|) and the codes t = clip(rint(w / s), -1, 1) (s = 0:
+    t = 0).  Returns (codes int8 [N, K], scales fp16 [N, K/128])."""
+    w = np.atleast_2d(np.asarray(w, dtype=np.float64))
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    codes = np.zeros((n, k), dtype=np.int8)
+    scales = np.zeros((n, k // GROUP), dtype=np.float16)
+    for r in range(n):
+        for g in range(k // GROUP):
+            grp = w[r, g * GROUP:(g + 1) * GROUP]
+            s = np.float16(np.mean(np.abs(grp)))
+            scales[r, g] = s
+            if s == 0:
+                continue
+            q = np.rint(grp / np.float64(s))
+            codes[r, g * GROUP:(g + 1) * GROUP] = np.clip(q, -1, 1).astype(np.int8)
+    return codes, scales
+
+
+def prepare_weights(w: np.ndarray, signs: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """The producer side of the layer: fold the rotation into a dense W, then
+    round to ternary g128 (codes, scales) for ``linear`` with these signs."""
+    return ternarize(fold_weights(w, signs))
+
 
 def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """w[n, k] = float64(s[n, k // 128]) * t[n, k]."""

@@ -143,6 +143,81 @@ def test_fold_invariant():
     assert np.abs(lhs - rhs).max() < 1e-11 * np.abs(rhs).max()
 
 
+def test_fold_weights_definition_matches_row_transform():
+    """W R block by block equals applying R^T to every row (the fold invariant's
+    form), and (R^T x) . (W R)^T = x . W^T."""
+    rng = np.random.default_rng(16)
+    k, n = 2048, 16
+    d = inputs.draw_signs(rng, k)
+    w = rng.standard_normal((n, k))
+    x = rng.standard_normal((2, k))
+    wf = orc.fold_weights(w, d)
+    assert np.abs(wf - orc.rotate(w, d)).max() < 1e-12
+    assert np.abs(orc.rotate(x, d) @ wf.T - x @ w.T).max() < 1e-11 * np.abs(x @ w.T).max()
+
+
+# ----------------------------------------------------------------- producer side
+
+def test_ternarize_worked_groups(golden):
+    rows = golden("ternarize_groups.txt")
+    for r in rows:
+        bar1, bar2 = r.index("|"), r.index("|", r.index("|") + 1)
+        pat = np.array([float(v) for v in r[:bar1]])
+        want_s = float(r[bar1 + 1])
+        want_t = np.array([int(v) for v in r[bar2 + 1:]], dtype=np.int8)
+        codes, scales = orc.ternarize(np.tile(pat, 32)[None, :])
+        assert scales.dtype == np.float16 and float(scales[0, 0]) == want_s, (pat, scales[0, 0])
+        assert np.array_equal(codes[0], np.tile(want_t, 32)), (pat, codes[0, :4])
+
+
+def test_ternarize_recovers_scaled_ternary_groups():
+    """w = c * t per group (t ternary with a fraction f of nonzeros, c > 0):
+    mean |w| = c f, every |w / s| is 0 or 1 / f >= 1, so the codes come back
+    exactly and the scale is fp16(c f)."""
+    rng = np.random.default_rng(17)
+    n, k = 6, 1024
+    t = inputs.draw_codes(rng, n, k, 0.4)
+    t[0, :128] = 0  # an all-zero group
+    c = np.exp2(rng.integers(-6, 3, size=(n, k // 128))).astype(np.float64)
+    w = t * np.repeat(c, 128, axis=1)
+    codes, scales = orc.ternarize(w)
+    assert np.array_equal(codes, t)
+    f = np.abs(t).reshape(n, k // 128, 128).mean(axis=2)
+    assert np.array_equal(scales, (c * f).astype(np.float16))
+    assert scales[0, 0] == 0
+
+
+def test_ternarize_symmetries():
+    rng = np.random.default_rng(18)
+    w = rng.standard_normal((4, 512))
+    codes, scales = orc.ternarize(w)
+    c2, s2 = orc.ternarize(-w)
+    assert np.array_equal(c2, -codes) and np.array_equal(s2, scales)
+    c3, s3 = orc.ternarize(8.0 * w)  # a power of two: every fp16 scale scales exactly
+    assert np.array_equal(c3, codes) and np.array_equal(s3, (8 * scales.astype(np.float64)).astype(np.float16))
+
+
+def test_prepare_weights_inverts_an_unfolded_ternary_layer():
+    """Start from ternary codes and power-of-two scales as the folded layer
+    W', unfold it (W = W' R^T), and prepare W: the fold must give W' back and
+    the rounding its codes and scales (all groups dense, so s = c exactly).  A
+    fold with R^T instead of R, or a missing sign, gives other codes."""
+    rng = np.random.default_rng(19)
+    n, k = 5, 2048
+    d = inputs.draw_signs(rng, k)
+    t = rng.choice(np.array([-1, 1], dtype=np.int8), size=(n, k))
+    s = np.exp2(rng.integers(-8, 0, size=(n, k // 128))).astype(np.float16)
+    w_folded = orc.dequantize(t, s)
+    w = orc.rotate(w_folded, d, inverse=True)  # rows times R^T: W = W' R^T
+    codes, scales = orc.prepare_weights(w, d)
+    assert np.array_equal(codes, t) and np.array_equal(scales, s)
+    x = rng.standard_normal((2, k))
+    y = orc.linear(x, codes, scales, d)
+    assert np.abs(y - x @ w.T).max() < 1e-10 * np.abs(x @ w.T).max()
+    wrong, _ = orc.ternarize(orc.rotate(w, d, inverse=True))  # folded with R^T
+    assert not np.array_equal(wrong, t)
+
+
 # ----------------------------------------------------------------- linear
 
 def test_linear_hand_computed(golden):
