@@ -1,4 +1,5 @@
-// Decode GEMV (M <= 4 tokens) on the tensor cores, 2-bit slot format.
+// Decode GEMV (M <= 16 tokens) on the tensor cores, 2-bit slot format (base-3
+// weights reach it after re-encoding to 2-bit slots).
 //
 // y[m, n] = sum_g s[n, g] * sum_{k in g} t[n, k] x'[m, k]   (ternary g128;
 // news.ditty.ir second paragraph; ai4coding.ru "What is a ternary model").
@@ -10,8 +11,9 @@
 // Those sums are tcgen05 kind::i8 MMAs: A = the codes c (u8) of 128 weight
 // rows, written by the unpacking threads straight into tensor memory (A from
 // TMEM: no shared-memory round trip for the big operand); B = the activation
-// planes (s8) of one group, 16 rows x 128 bytes in shared memory (row 2m = hi
-// and 2m + 1 = lo of token m, the rest zero); D = int32 in TMEM.  One group per MMA chain, so
+// planes (s8) of one group, 16 rows (up to 8 tokens) or 32 rows (up to 16) x
+// 128 bytes in shared memory (row 2m = hi and 2m + 1 = lo of token m, the rest
+// zero); D = int32 in TMEM.  One group per MMA chain, so
 // each D holds exact per-group sums that the same threads read back and scale
 // by s[n, g] * e_g in fp32.
 //
