@@ -36,6 +36,11 @@ Readings taken where the pages are silent (each is stated again in the design doc):
   A byte >= 243, or a last byte whose digits 3 and 4 are not both 1, is invalid:
   all codes it carries decode to t = 0 and it is counted once.
 * Codes outside {-1, 0, 1} given to the packer are packed as t = 0 and counted.
+* 1-bit g128 (dev.to, "How Prism ML Squeezed a 27B Model Into 3.9 GB", the
+  list of the two formats that ship: each weight -1 or +1 with one scale per
+  128 weights, about 1.125 bits): byte i of a row holds k = 8i..8i+7, weight
+  8i+j in bit j, bit 1 = +1 and bit 0 = -1.  Any other code given to the
+  packer (0 included) is packed as -1 and counted; every byte is valid.
 * Integer mode: y[m, n] = sum_k t[n, k] x[m, k] for int8 x, no scales, no rotation.
 * Producer side (openbonsai.org, "How it works", steps 1 "Rotate" and 2
   "Round"): the pages round with sequential GPTQ on calibration data, which
@@ -56,6 +61,7 @@ GROUP = 128
 BLOCK = 1024
 FMT_2BIT = "2bit"
 FMT_BASE3 = "base3"
+FMT_1BIT = "1bit"
 BASE3_GROUP_BYTES = 26
 
 
@@ -202,6 +208,8 @@ def packed_bytes(fmt: str, n: int, k: int) -> int:
         return n * (k // 4)
     if fmt == FMT_BASE3:
         return n * (k // GROUP) * BASE3_GROUP_BYTES
+    if fmt == FMT_1BIT:
+        return n * (k // 8)
     raise ValueError(f"unknown format {fmt!r}")
 
 
@@ -213,6 +221,11 @@ def pack(codes: np.ndarray, fmt: str) -> tuple[np.ndarray, int]:
     """Pack int8 codes [N, K] -> (uint8 [N, row_bytes], invalid code count)."""
     t = np.asarray(codes).astype(np.int64)
     n, k = t.shape
+    if fmt == FMT_1BIT:
+        ok1 = (t == -1) | (t == 1)
+        bit = (t == 1).astype(np.int64).reshape(n, k // 8, 8)
+        byte = sum(bit[..., j] << j for j in range(8))
+        return byte.astype(np.uint8), int((~ok1).sum())
     ok = _valid_code_mask(t)
     invalid = int((~ok).sum())
     c = np.where(ok, t + 1, 1)  # biased code, invalid -> t = 0
@@ -235,6 +248,11 @@ def pack(codes: np.ndarray, fmt: str) -> tuple[np.ndarray, int]:
 def unpack(packed: np.ndarray, fmt: str, n: int, k: int) -> tuple[np.ndarray, int]:
     """Unpack uint8 [N, row_bytes] -> (int8 codes [N, K], invalid count)."""
     p = np.asarray(packed).astype(np.int64).reshape(n, -1)
+    if fmt == FMT_1BIT:
+        if p.shape[1] != k // 8:
+            raise ValueError("row bytes must be K/8")
+        bits = np.stack([(p >> j) & 1 for j in range(8)], axis=-1).reshape(n, k)
+        return (2 * bits - 1).astype(np.int8), 0
     if fmt == FMT_2BIT:
         if p.shape[1] != k // 4:
             raise ValueError("row bytes must be K/4")

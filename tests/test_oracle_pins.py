@@ -408,6 +408,40 @@ def test_pack_counts_invalid_codes(fmt):
     assert bad2 == 0 and np.all(back == 0)
 
 
+def test_pack_1bit_worked_bytes(golden):
+    for r in golden("pack_1bit.txt"):
+        byte = int(r[0], 16)
+        want = np.array([int(v) for v in r[1:]], dtype=np.int8)
+        codes, bad = orc.unpack(np.array([[byte]] * 16, dtype=np.uint8).reshape(1, 16), "1bit", 1, 128)
+        assert bad == 0 and np.array_equal(codes[0, :8], want), (hex(byte), codes[0, :8])
+        packed, bad = orc.pack(np.tile(want, 16)[None, :], "1bit")
+        assert bad == 0 and np.all(packed == byte)
+
+
+def test_pack_1bit_round_trip_and_invalid_codes():
+    rng = np.random.default_rng(50)
+    t = rng.choice(np.array([-1, 1], dtype=np.int8), size=(7, 1024))
+    packed, bad = orc.pack(t, "1bit")
+    assert bad == 0 and packed.shape == (7, 128) and orc.packed_bytes("1bit", 7, 1024) == 7 * 128
+    back, bad = orc.unpack(packed, "1bit", 7, 1024)
+    assert bad == 0 and np.array_equal(back, t)
+    # every one of the 256 byte values is a valid code byte and comes back
+    allb = np.arange(256, dtype=np.uint8)[None, :].repeat(1, 0).reshape(1, 256)
+    codes, bad = orc.unpack(np.tile(allb, (1, 4)), "1bit", 1, 8192)
+    assert bad == 0 and set(np.unique(codes)) == {-1, 1}
+    again, _ = orc.pack(codes, "1bit")
+    assert np.array_equal(again, np.tile(allb, (1, 4)))
+    # zeros and out-of-range codes are counted and packed as -1
+    t2 = t.copy()
+    t2[0, :3] = [0, 2, -5]
+    p2, bad2 = orc.pack(t2, "1bit")
+    assert bad2 == 3
+    back2, _ = orc.unpack(p2, "1bit", 7, 1024)
+    assert np.all(back2[0, :3] == -1)
+    # the pages' ~1.125 bits per weight for 1-bit g128, as this layout's arithmetic
+    assert orc.bits_per_weight("1bit") == 1.125
+
+
 def test_bits_per_weight_arithmetic():
     n, k = 17408, 5120
     assert orc.packed_bytes("2bit", n, k) * 8 / (n * k) + 16 / 128 == 2.125
