@@ -98,7 +98,11 @@ typedef int tb_path;
                             of 4 tokens).  One token (2-bit): one launch that
                             rotates x itself for K <= 8192                     */
 #define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
-                            s*t in shared memory, fp32 accumulators in TMEM)    */
+                            s*t in shared memory, fp32 accumulators in TMEM);
+                            base-3 from 8 tokens, re-encoded to 2-bit slots in
+                            the workspace first.  Chosen by TB_PATH_AUTO past
+                            16 tokens, or from 8 base-3 tokens when N is above
+                            the tensor-core decode's 148 * 128 rows            */
 #define TB_PATH_SIMPLE 3 /* plain per-row kernel: any K % 128, any alignment    */
 #define TB_PATH_GEMV_TC 4 /* tcgen05 decode kernel (codes unpacked into TMEM as
                             the u8 A operand, int8 activation planes as B in
@@ -179,7 +183,8 @@ tb_status tb_ternary_linear(const void* x, tb_dtype xt, const uint8_t* packed,
  * 16-byte aligned packed/scales; GEMV_TC needs float mode, M <= 16 (base-3:
  * 8 <= M <= 16), K % 1024 == 0, aligned pointers and a plan that fits the
  * SMs; GEMM needs float mode, K % 1024 == 0 and aligned pointers (base-3:
- * M > 16); SIMPLE takes everything tb_ternary_linear takes. */
+ * M >= 8, re-encoded to 2-bit slots in the workspace first); SIMPLE takes
+ * everything tb_ternary_linear takes. */
 tb_status tb_ternary_linear_ex(const void* x, tb_dtype xt, const uint8_t* packed,
                                const uint16_t* scales, tb_format f, int64_t M, int64_t N,
                                int64_t K, const int8_t* signs, void* y, tb_dtype yt,

@@ -480,8 +480,10 @@ bool gemv_tc_ok(const LinearArgs& a) {
 }
 
 bool gemm_ok(const LinearArgs& a) {
-  // base-3 is served by re-encoding to 2-bit slots first (more than 16 tokens)
-  if (a.f == TB_FMT_BASE3 && a.M <= 16) return false;
+  // base-3 is served by re-encoding to 2-bit slots first, which the workspace
+  // holds from kB3TranscodeMinM tokens on (up to 16 tokens the tensor-core
+  // decode comes first where its row limit allows)
+  if (a.f == TB_FMT_BASE3 && a.M < kB3TranscodeMinM) return false;
   return is_float_dtype(a.xt) && a.K % 1024 == 0 && fast_aligned(a) &&
          (a.M + kGemmUM - 1) / kGemmUM <= 65535 && a.N < (int64_t(1) << 30);
 }

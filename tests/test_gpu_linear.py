@@ -236,12 +236,20 @@ def test_gemm_2bit(case):
     _check(prob.linear(GEMM), ref, prob.p)
 
 
-@pytest.mark.parametrize("m", [17, 300])
+@pytest.mark.parametrize("m", [8, 12, 17, 300])
 def test_gemm_base3_via_reencoding(m):
     """Base-3 prefill: the weights are re-encoded to 2-bit slots in the
     workspace, then the tensor-core GEMM runs on them."""
     prob, ref = _problem(27, m, 1001, 2048, 0.33, "base3", "abs_normal", 0.01)
     _check(prob.linear(GEMM), ref, prob.p)
+    _check(prob.linear(AUTO), ref, prob.p)
+
+
+def test_base3_tokens_beyond_tensor_core_rows_take_the_gemm():
+    """12 base-3 tokens and more rows than the tensor-core decode takes: the
+    automatic path re-encodes to 2-bit slots and runs the GEMM."""
+    assert tb.tb_ternary_linear_path(tb.TB_BF16, "base3", 12, 19000, 1024, True, True) == GEMM
+    prob, ref = _problem(28, 12, 19000, 1024, 0.33, "base3", "abs_normal", 0.01)
     _check(prob.linear(AUTO), ref, prob.p)
 
 
