@@ -1,12 +1,14 @@
 """Benchmark of the ternary-g128 linear layer (signed block-Hadamard rotation
 folded into the weights) on B200.
 
-A step is one call of tb_ternary_linear on the decode GEMV workload
-(M=1, K=5120, N=17408, ternary codes with P(0)=0.33, fp16 g128 scales, bf16
-activations with 1% outliers): the inverse rotation of the activations and the
-packed-weight GEMV.  The metric is packed-weight GB/s (codes + scales read
-once per step).  Successive steps read successive copies of the weights, and
-the copies together are larger than L2, so every step streams from HBM.
+The workload is the decode GEMV (M=1, K=5120, N=17408, ternary codes with
+P(0)=0.33, fp16 g128 scales, bf16 activations with 1% outliers).  One call of
+tb_ternary_linear is one pass of the hot path: the inverse rotation of the
+activations and the packed-weight GEMV.  A step is a fixed batch of
+CALLS_PER_STEP such calls, back to back in one CUDA graph, successive calls on
+successive copies of the weights (together larger than L2, so every call
+streams its weights from HBM).  `--steps K` times exactly K steps.  The metric
+is packed-weight GB/s (codes + scales read once per call).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--fmt 2bit|base3]
   python bench.py --impl reference ...   (the CPU oracle on the same workload)
@@ -35,6 +37,8 @@ WORKLOAD = "gemv_gateup_k5120_n17408"
 METRIC = "ternary-g128 GEMV packed-weight GB/s vs HBM peak (M=1); prefill GEMM tok/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
+CALLS_PER_STEP = 1000   # decode calls per step (rounded up to whole rounds of the weight copies)
+PREFILL_CALLS_PER_STEP = 24  # prefill calls per step (a multiple of its 6 weight copies)
 
 
 def _barrier(world):
@@ -180,9 +184,38 @@ def _upload_problem(tb, inputs, dev, fmt, m, n, k, seed, p0, scale_kind, outlier
     return p, packs, scls, x, signs
 
 
+def _timed_replays(graph, steps, stream, dev, world):
+    """Replays `graph` exactly `steps` times between a barrier and a device
+    synchronisation on both sides; CUDA events on the launching stream give
+    the total (max over ranks) and each replay's own time."""
+    import torch
+    _barrier(world)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    with torch.cuda.stream(stream):
+        ev[0].record(stream)
+        for i in range(steps):
+            graph.replay()
+            ev[i + 1].record(stream)
+    ev[-1].synchronize()
+    torch.cuda.synchronize()
+    _barrier(world)
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total = _max_over_ranks(ev[0].elapsed_time(ev[-1]), dev, world)
+    return total, per
+
+
+def _spread(per, calls):
+    """Median, p10 and p90 of the per-call time over the timed steps (ms)."""
+    v = sorted(x / calls for x in per)
+    q = lambda f: v[min(len(v) - 1, int(round(f * (len(v) - 1))))]
+    return {"median": round(q(0.5), 6), "p10": round(q(0.1), 6), "p90": round(q(0.9), 6)}
+
+
 def measure_decode(args, tb, inputs, dev, stream, fmt, m, n, k, seed, p0, scale_kind, outlier, world, sample=True):
-    """Device time per call of tb_ternary_linear on the decode workload, calls
-    back to back in CUDA graphs, successive calls on successive weight copies
+    """Device time of `args.steps` steps of back-to-back tb_ternary_linear
+    calls on the decode workload: a step is one replay of a CUDA graph of
+    about CALLS_PER_STEP calls, successive calls on successive weight copies
     (together larger than L2, so every call streams its weights from HBM)."""
     import torch
     step_bytes = _packed_bytes(fmt, n, k)
@@ -194,49 +227,34 @@ def measure_decode(args, tb, inputs, dev, stream, fmt, m, n, k, seed, p0, scale_
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     sh = stream.cuda_stream
 
-    def step(i):
+    def call(i):
         j = i % copies
         tb.tb_ternary_linear(x, tb.TB_BF16, packs[j], scls[j], fmt, m, n, k, signs, y, tb.TB_FP32, ws, ws_bytes,
                              stream=sh)
 
-    chunk = min(args.steps, 1200)
-    chunk -= chunk % copies if chunk >= copies else 0
-    chunk = max(chunk, 1)
+    calls = copies * int(np.ceil(CALLS_PER_STEP / copies))
     with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
-            step(i)
+        for i in range(copies):
+            call(i)
     stream.synchronize()
     g_main = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g_main, stream=stream):
-            for i in range(chunk):
-                step(i)
-        for _ in range(2):
+            for i in range(calls):
+                call(i)
+        for _ in range(args.warmup):  # warm-up steps (untimed)
             g_main.replay()
     stream.synchronize()
-    reps = max(1, args.steps // chunk)
     sampler = ClockSampler(torch.cuda.current_device()) if sample else None
     if sampler:
         sampler.start()
-    _barrier(world)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(reps):
-            g_main.replay()
-        e1.record(stream)
-    e1.synchronize()
-    torch.cuda.synchronize()
-    _barrier(world)
-    ms = _max_over_ranks(e0.elapsed_time(e1), dev, world)
+    ms, per = _timed_replays(g_main, args.steps, stream, dev, world)
     clocks = sampler.stop() if sampler else None
     del g_main
-    steps = reps * chunk
-    return {"ms_per_step": ms / steps, "steps": steps, "step_bytes": step_bytes, "copies": copies,
-            "path": tb.tb_ternary_linear_path(tb.TB_BF16, fmt, m, n, k, True, True),
-            "launches": _launches_per_call(tb, fmt, m, n, k) * steps, "clocks": clocks,
+    return {"ms_per_call": ms / (args.steps * calls), "ms_per_step": ms / args.steps, "steps": args.steps,
+            "calls_per_step": calls, "per_call_spread": _spread(per, calls), "step_bytes": step_bytes,
+            "copies": copies, "path": tb.tb_ternary_linear_path(tb.TB_BF16, fmt, m, n, k, True, True),
+            "launches": _launches_per_call(tb, fmt, m, n, k) * calls * args.steps, "clocks": clocks,
             "problem": (p, packs, scls, x, signs, ws, ws_bytes, copies)}
 
 
@@ -280,7 +298,7 @@ def measure_e2e(args, tb, dev, stream, fmt, m, n, k, prob, world):
         stream.wait_stream(s_in)
         stream.wait_stream(s_out)
 
-    chunk = 2 * copies * max(1, 240 // (2 * copies))
+    calls = 2 * copies * int(np.ceil(CALLS_PER_STEP / (2 * copies)))
     with torch.cuda.stream(stream):
         steps(2 * copies)
     torch.cuda.synchronize()
@@ -291,38 +309,28 @@ def measure_e2e(args, tb, dev, stream, fmt, m, n, k, prob, world):
         with torch.cuda.graph(g, stream=stream):
             s_in.wait_stream(stream)
             s_out.wait_stream(stream)
-            steps(chunk)
-        g.replay()
-    torch.cuda.synchronize()
-    reps = max(1, min(args.steps, 20 * chunk) // chunk)
-    _barrier(world)
-    torch.cuda.synchronize()
-    a0 = torch.cuda.Event(enable_timing=True)
-    a1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        a0.record(stream)
-        for _ in range(reps):
+            steps(calls)
+        for _ in range(args.warmup):
             g.replay()
-        a1.record(stream)
-    a1.synchronize()
     torch.cuda.synchronize()
-    _barrier(world)
-    ms = _max_over_ranks(a0.elapsed_time(a1), dev, world)
+    ms, per = _timed_replays(g, args.steps, stream, dev, world)
     del g
-    e2e_ms = ms / (reps * chunk)
+    e2e_ms = ms / (args.steps * calls)
     step_bytes = _packed_bytes(fmt, n, k)
     return {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": int(m * k * 2), "d2h_bytes_per_step": int(m * n * 4),
-            "ms_per_step": round(e2e_ms, 5), "steps": reps * chunk,
-            "how": "CUDA graph; per step: pinned-host x -> device, tb_ternary_linear, device y -> pinned host; "
-                   "copies and compute of consecutive steps overlap on three streams, two buffer sets"}
+            "h2d_bytes_per_step": int(calls * m * k * 2), "d2h_bytes_per_step": int(calls * m * n * 4),
+            "calls_per_step": calls, "ms_per_call": round(e2e_ms, 6), "ms_per_step": round(ms / args.steps, 4),
+            "steps": args.steps, "per_call_spread": _spread(per, calls),
+            "how": "CUDA graph per step; per call: pinned-host x -> device, tb_ternary_linear, device y -> pinned "
+                   "host; copies and compute of consecutive calls overlap on three streams, two buffer sets"}
 
 
 def _decode_entry(res, peak, peak_kind, world):
-    gbs = res["step_bytes"] / (res["ms_per_step"] * 1e-3) / 1e9
-    return {"value": round(gbs * world, 2), "unit": "GB/s", "ms_per_step": round(res["ms_per_step"], 6),
-            "bytes_per_step": res["step_bytes"], "steps": res["steps"], "kernel_path": res["path"],
-            "weight_copies": res["copies"],
+    gbs = res["step_bytes"] / (res["ms_per_call"] * 1e-3) / 1e9
+    return {"value": round(gbs * world, 2), "unit": "GB/s", "ms_per_call": round(res["ms_per_call"], 6),
+            "ms_per_step": round(res["ms_per_step"], 4), "calls_per_step": res["calls_per_step"],
+            "per_call_spread": res["per_call_spread"], "bytes_per_call": res["step_bytes"], "steps": res["steps"],
+            "kernel_path": res["path"], "weight_copies": res["copies"],
             "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(gbs / peak, 4),
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
@@ -359,12 +367,15 @@ def run_ours(args, rank, world):
         res.pop("problem")
         torch.cuda.empty_cache()
     prefill = run_prefill(args, dev, stream, tb, inputs, world) if args.prefill else None
+    stack = (stack_cells(args, dev, stream, tb, inputs, ["2bit"], [1, 16], [0.33], ["separate", "shared_input"],
+                         args.steps, inputs.STACK_LAYERS, world) if args.stack_leg else None)
     head = _decode_entry(main, peak, peak_kind, world)
     roof = head["roofline"]
     roof["traffic"] = _traffic(args.fmt)
     roof["kernel"] = ("tb_ternary_linear decode call (gemv1_2bit_kernel, rotation fused)" if args.fmt == "2bit"
                       else "tb_ternary_linear decode call (prep_b3_kernel + gemv_b3_kernel)")
-    roof["timing"] = "device time per call of back-to-back calls in CUDA graphs (CUDA events on the launching stream)"
+    roof["timing"] = ("device time per call over the timed steps (back-to-back calls in a CUDA graph, CUDA events "
+                      "on the launching stream)")
     return {
         "metric": METRIC,
         "value": head["value"],
@@ -381,7 +392,8 @@ def run_ours(args, rank, world):
         "data": "synthetic (seeded; codes P(0)=0.33, |N(0,1)|*0.02 fp16 scales, N(0,1) bf16 x with 1% +-20 outliers)",
         "config": {"workload": f"decode GEMV gate/up M=1 K=5120 N=17408 ({args.fmt} packing)",
                    "M": m, "K": k, "N": n, "format": args.fmt, "kernel_path": main["path"],
-                   "bytes_per_step": main["step_bytes"], "weight_copies": main["copies"],
+                   "calls_per_step": main["calls_per_step"], "bytes_per_call": main["step_bytes"],
+                   "weight_copies": main["copies"],
                    "l2": f"inputs larger than L2: {main['copies']} weight copies, "
                          f"{main['copies'] * main['step_bytes'] / 1e6:.0f} MB > 126 MB",
                    "parallelism": f"replicas x{world}"},
@@ -389,6 +401,7 @@ def run_ours(args, rank, world):
         "formats": others,
         "e2e": e2e,
         "prefill": prefill,
+        "stack": stack,
         "gpu_launches": main["launches"],
         "clocks": main["clocks"],
     }
@@ -398,21 +411,23 @@ def run_prefill(args, dev, stream, tb, inputs, world=1):
     """Prefill GEMM workload (M=2048 tokens, K=5120, N=17408, 2-bit): tokens/s
     of the whole job (every rank one replica, timed as the slowest rank),
     TFLOP-equivalent/s per GPU (2*M*N*K per call) and its fraction of the
-    measured dense 16-bit tensor peak.  Two weight copies alternate; the call
-    is compute-bound."""
+    measured dense 16-bit tensor peak.  Successive calls take successive
+    copies of the weights (6) and of the activations (2), 185 MB together,
+    more than L2; the call is compute-bound."""
     import torch
 
     w = inputs.WORKLOADS["prefill_m2048_k5120_n17408"]
     m, n, k = 2048, w["n"], w["k"]
     p = inputs.make_linear_inputs(w["seed"], m, n, k, w["p0"])
     codes = torch.from_numpy(p.codes).to(dev)
+    wcopies, xcopies = 6, 2
     packs = [torch.empty(tb.tb_packed_bytes("2bit", n, k), dtype=torch.uint8, device=dev)
-             for _ in range(2)]
+             for _ in range(wcopies)]
     for pk in packs:
         tb.tb_pack_ternary("2bit", codes, n, k, pk)
     del codes
-    scales = torch.from_numpy(p.scales.view(np.int16)).to(dev)
-    x = torch.from_numpy(p.x_bf16.view(np.int16)).to(dev).view(torch.bfloat16)
+    scls = [torch.from_numpy(p.scales.view(np.int16)).to(dev) for _ in range(wcopies)]
+    xs = [torch.from_numpy(p.x_bf16.view(np.int16)).to(dev).view(torch.bfloat16) for _ in range(xcopies)]
     signs = torch.from_numpy(p.signs).to(dev)
     y = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
     ws_bytes = tb.tb_ternary_linear_workspace("2bit", m, n, k)
@@ -420,40 +435,38 @@ def run_prefill(args, dev, stream, tb, inputs, world=1):
     sh = stream.cuda_stream
 
     def call(i):
-        tb.tb_ternary_linear(x, tb.TB_BF16, packs[i % 2], scales, "2bit", m, n, k, signs, y,
-                             tb.TB_BF16, ws, ws_bytes, stream=sh)
+        tb.tb_ternary_linear(xs[i % xcopies], tb.TB_BF16, packs[i % wcopies], scls[i % wcopies], "2bit", m, n, k,
+                             signs, y, tb.TB_BF16, ws, ws_bytes, stream=sh)
 
-    steps = max(10, min(200, args.steps // 100))
+    calls = PREFILL_CALLS_PER_STEP
     with torch.cuda.stream(stream):
-        for i in range(5):
+        for i in range(3):
             call(i)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            for i in range(steps):
+            for i in range(calls):
                 call(i)
-        g.replay()
+        for _ in range(args.warmup):
+            g.replay()
     stream.synchronize()
-    _barrier(world)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-    e1.synchronize()
-    torch.cuda.synchronize()
-    _barrier(world)
-    ms = _max_over_ranks(e0.elapsed_time(e1), dev, world) / steps
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    total, per = _timed_replays(g, args.steps, stream, dev, world)
+    clocks = sampler.stop()
+    del g
+    ms = total / (args.steps * calls)
     flops = 2.0 * m * n * k
     tflops = flops / (ms * 1e-3) / 1e12
     peak, kind = _tensor_peak()
     return {"workload": "prefill GEMM M=2048 K=5120 N=17408 (2bit), bf16 in/out",
-            "tok_s": round(m * world / (ms * 1e-3), 1), "ms_per_call": round(ms, 5), "steps": steps,
-            "tflops_equiv": round(tflops, 2),
+            "tok_s": round(m * world / (ms * 1e-3), 1), "ms_per_call": round(ms, 5),
+            "calls_per_step": calls, "steps": args.steps, "ms_timed": round(total, 3),
+            "l2": "6 weight copies and 2 activation copies in rotation, 185 MB > 126 MB L2",
+            "per_call_spread": _spread(per, calls), "tflops_equiv": round(tflops, 2),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
                          "peak_source": kind, "dtype": "fp16 x fp16 -> fp32 (kind::f16)"},
+            "clocks": clocks,
             "kernel_path": tb.tb_ternary_linear_path(tb.TB_BF16, "2bit", m, n, k, True, True)}
 
 
@@ -522,20 +535,116 @@ def run_sweep(args, rank, world):
                                  w["scale_kind"], w["outlier_rate"], world, sample=False)
             res.pop("problem")
             e = _decode_entry(res, peak, peak_kind, world)
-            e.update({"format": fmt, "M": m, "tokens_per_s": round(m / (res["ms_per_step"] * 1e-3), 1)})
+            e.update({"format": fmt, "M": m, "tokens_per_s": round(m / (res["ms_per_call"] * 1e-3), 1)})
             cells.append(e)
             torch.cuda.empty_cache()
     return {"sweep": "decode GEMV down K=17408 N=5120", "cells": cells}
 
 
+STACK_CALLS = {
+    # one call per matrix: 7 calls (7 rotations) per layer
+    "separate": (("q",), ("k",), ("v",), ("o",), ("gate",), ("up",), ("down",)),
+    # one call per shared input: q|k|v and gate|up stacked along N, 4 calls
+    # (4 rotations) per layer
+    "shared_input": (("q", "k", "v"), ("o",), ("gate", "up"), ("down",)),
+}
+
+
+def stack_cells(args, dev, stream, tb, inputs, fmts, ms, p0s, modes, steps, layers, world=1):
+    """The synthetic 27B-class layer stack: `layers` layers x {q, k, v, o,
+    gate, up, down} of distinct ternary weights (5.8 GB in 2-bit slots, 4.8 GB
+    in base-3 at 64 layers).  One pass = every call of the stack in one CUDA
+    graph; every call reads the synthetic input of its width (no attention or
+    nonlinearity between the linears).  Calls per layer: 7 (mode "separate") or
+    4 (mode "shared_input": matrices that read the same input stacked along N
+    behind one rotation).  `steps` passes are timed (a pass reads the whole
+    stack, far more than L2).  Per cell: device time per pass, tokens/s =
+    M / time, packed-weight GB/s."""
+    import torch
+
+    seed = 4
+    shapes = {name: (n, k) for name, n, k in inputs.STACK_LAYER_SHAPES}
+    mat = {name: j for j, (name, _, _) in enumerate(inputs.STACK_LAYER_SHAPES)}
+    peak, peak_kind = _peaks()
+    kdims = sorted({k for _, k in shapes.values()})
+    xin = {}
+    for m in ms:
+        for k in kdims:
+            xb, sg = inputs.stack_activations(seed, m, k)
+            xin[(m, k)] = (torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16),
+                           torch.from_numpy(sg).to(dev))
+    cells = []
+    for p0 in p0s:
+        for f in fmts:
+            # every matrix generated once and packed into the buffer of its
+            # call in each mode
+            bufs = {mode: [] for mode in modes}
+            for layer in range(layers):
+                where = {}
+                for mode in modes:
+                    for names in STACK_CALLS[mode]:
+                        k = shapes[names[0]][1]
+                        ntot = sum(shapes[nm][0] for nm in names)
+                        pk = torch.empty(tb.tb_packed_bytes(f, ntot, k), dtype=torch.uint8, device=dev)
+                        sc = torch.empty(ntot, k // 128, dtype=torch.int16, device=dev)
+                        bufs[mode].append((pk, sc, ntot, k))
+                        row = 0
+                        for nm in names:
+                            where.setdefault(nm, []).append((pk, sc, row))
+                            row += shapes[nm][0]
+                for nm, (n, k) in shapes.items():
+                    codes = inputs.stack_codes_torch(seed, layer, mat[nm], n, k, p0, dev)
+                    scn = torch.from_numpy(inputs.stack_scales(seed, layer, mat[nm], n, k).view(np.int16)).to(dev)
+                    rb = tb.tb_packed_bytes(f, 1, k)
+                    for pk, sc, row in where[nm]:
+                        tb.tb_pack_ternary(f, codes, n, k, pk[row * rb:(row + n) * rb])
+                        sc[row:row + n].copy_(scn)
+                    del codes
+            torch.cuda.synchronize()
+            pass_bytes = sum(_packed_bytes(f, n, k) for n, k in shapes.values()) * layers
+            for mode in modes:
+                for m in ms:
+                    ns = {b[2] for b in bufs[mode]}
+                    ys = {n: torch.empty(m, n, dtype=torch.float32, device=dev) for n in ns}
+                    wsb = max(tb.tb_ternary_linear_workspace(f, m, b[2], b[3]) for b in bufs[mode])
+                    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+                    sh = stream.cuda_stream
+                    paths = sorted({tb.tb_ternary_linear_path(tb.TB_BF16, f, m, b[2], b[3], True, True)
+                                    for b in bufs[mode]})
+
+                    def one_pass():
+                        for pk, sc, n, k in bufs[mode]:
+                            x, sg = xin[(m, k)]
+                            tb.tb_ternary_linear(x, tb.TB_BF16, pk, sc, f, m, n, k, sg, ys[n], tb.TB_FP32, ws, wsb,
+                                                 stream=sh)
+
+                    with torch.cuda.stream(stream):
+                        one_pass()
+                        g = torch.cuda.CUDAGraph()
+                        with torch.cuda.graph(g, stream=stream):
+                            one_pass()
+                        for _ in range(max(1, args.warmup)):
+                            g.replay()
+                    stream.synchronize()
+                    total, per = _timed_replays(g, steps, stream, dev, world)
+                    ms_pass = total / steps
+                    gbs = pass_bytes / (ms_pass * 1e-3) / 1e9
+                    cells.append({"format": f, "p0": p0, "M": m, "mode": mode, "ms_per_pass": round(ms_pass, 4),
+                                  "tokens_per_s": round(world * m / (ms_pass * 1e-3), 1),
+                                  "weight_GBs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4),
+                                  "paths": paths, "calls_per_pass": len(bufs[mode]), "passes_timed": steps})
+                    del g, ws, ys
+                    torch.cuda.empty_cache()
+            del bufs
+            torch.cuda.empty_cache()
+    return {"stack": f"synthetic 27B-class layer stack, {layers} layers x 7 linears",
+            "bytes_per_pass": {f: sum(_packed_bytes(f, n, k) for n, k in shapes.values()) * layers for f in fmts},
+            "peak_GBs": peak, "peak_source": peak_kind, "cells": cells}
+
+
 def run_stack(args, rank, world):
-    """The synthetic 27B-class layer stack: 64 layers x {q, k, v, o, gate, up,
-    down} of distinct ternary weights (5.8 GB in 2-bit slots, 4.8 GB in base-3),
-    M in {1, 4, 16, 64, 512} tokens, zero fraction in {0.2, 0.33, 0.5}, both
-    packings.  One pass = the 448 tb_ternary_linear calls of the stack, captured
-    in one CUDA graph; every linear reads its own synthetic input (no attention
-    or nonlinearity between them).  Reported per cell: device time per pass,
-    tokens/s = M / time, and packed-weight GB/s.  Printed as its own JSON line."""
+    """The stack sweep (--stack): every (zero fraction, packing, call mode,
+    tokens) cell asked for.  Printed as its own JSON line."""
     import torch
 
     from ternary_weight_signed_b200 import binding as tb
@@ -547,82 +656,9 @@ def run_stack(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(device=dev)
-    seed = 4
-    layers = args.stack_layers
-    shapes = inputs.STACK_LAYER_SHAPES
-    ms = [int(v) for v in args.stack_ms.split(",")]
-    p0s = [float(v) for v in args.stack_p0.split(",")]
-    fmts = args.stack_fmts.split(",")
-    peak, peak_kind = _peaks()
-    kdims = sorted({k for _, _, k in shapes})
-    xin = {}
-    for m in ms:
-        for k in kdims:
-            xb, sg = inputs.stack_activations(seed, m, k)
-            xin[(m, k)] = (torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16),
-                           torch.from_numpy(sg).to(dev))
-    cells = []
-    for p0 in p0s:
-        t_gen = time.perf_counter()
-        weights = {f: [] for f in fmts}
-        scales = []
-        for layer in range(layers):
-            for j, (_, n, k) in enumerate(shapes):
-                codes = inputs.stack_codes_torch(seed, layer, j, n, k, p0, dev)
-                for f in fmts:
-                    pk = torch.empty(tb.tb_packed_bytes(f, n, k), dtype=torch.uint8, device=dev)
-                    tb.tb_pack_ternary(f, codes, n, k, pk)
-                    weights[f].append(pk)
-                del codes
-                scales.append(torch.from_numpy(inputs.stack_scales(seed, layer, j, n, k).view(np.int16)).to(dev))
-        torch.cuda.synchronize()
-        t_gen = time.perf_counter() - t_gen
-        for f in fmts:
-            pass_bytes = sum(_packed_bytes(f, n, k) for _, n, k in shapes) * layers
-            for m in ms:
-                ys = {n: torch.empty(m, n, dtype=torch.float32, device=dev) for n in {n for _, n, _ in shapes}}
-                wsb = max(tb.tb_ternary_linear_workspace(f, m, n, k) for _, n, k in shapes)
-                ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
-                sh = stream.cuda_stream
-                paths = sorted({tb.tb_ternary_linear_path(tb.TB_BF16, f, m, n, k, True, True) for _, n, k in shapes})
-
-                def one_pass():
-                    for layer in range(layers):
-                        for j, (_, n, k) in enumerate(shapes):
-                            x, sg = xin[(m, k)]
-                            idx = layer * len(shapes) + j
-                            tb.tb_ternary_linear(x, tb.TB_BF16, weights[f][idx], scales[idx], f, m, n, k, sg, ys[n],
-                                                 tb.TB_FP32, ws, wsb, stream=sh)
-
-                with torch.cuda.stream(stream):
-                    one_pass()
-                    g = torch.cuda.CUDAGraph()
-                    with torch.cuda.graph(g, stream=stream):
-                        one_pass()
-                    g.replay()
-                stream.synchronize()
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                reps = 3
-                with torch.cuda.stream(stream):
-                    e0.record(stream)
-                    for _ in range(reps):
-                        g.replay()
-                    e1.record(stream)
-                e1.synchronize()
-                ms_pass = e0.elapsed_time(e1) / reps
-                gbs = pass_bytes / (ms_pass * 1e-3) / 1e9
-                cells.append({"format": f, "p0": p0, "M": m, "ms_per_pass": round(ms_pass, 4),
-                              "tokens_per_s": round(m / (ms_pass * 1e-3), 1), "weight_GBs": round(gbs, 1),
-                              "hbm_frac": round(gbs / peak, 4), "paths": paths,
-                              "calls_per_pass": layers * len(shapes)})
-                del g, ws, ys
-                torch.cuda.empty_cache()
-        del weights, scales
-        torch.cuda.empty_cache()
-    return {"stack": f"synthetic 27B-class layer stack, {layers} layers x {len(shapes)} linears",
-            "bytes_per_pass": {f: sum(_packed_bytes(f, n, k) for _, n, k in shapes) * layers for f in fmts},
-            "peak_GBs": peak, "peak_source": peak_kind, "cells": cells}
+    return stack_cells(args, dev, stream, tb, inputs, args.stack_fmts.split(","),
+                       [int(v) for v in args.stack_ms.split(",")], [float(v) for v in args.stack_p0.split(",")],
+                       args.stack_modes.split(","), args.steps, args.stack_layers, world)
 
 
 def run_reference(args, rank, world):
@@ -662,8 +698,8 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--fmt", default="2bit", choices=["2bit", "base3"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -674,6 +710,9 @@ def main():
     ap.add_argument("--stack-ms", default="1,4,16,64,512")
     ap.add_argument("--stack-p0", default="0.2,0.33,0.5")
     ap.add_argument("--stack-fmts", default="2bit,base3")
+    ap.add_argument("--stack-modes", default="separate,shared_input")
+    ap.add_argument("--no-stack", dest="stack_leg", action="store_false",
+                    help="leave the layer-stack leg out of the bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

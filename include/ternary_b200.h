@@ -150,6 +150,28 @@ tb_status tb_hadamard_rotate(const void* x, tb_dtype xt, void* y, tb_dtype yt,
                              const int8_t* signs, int64_t M, int64_t K, int inverse,
                              void* stream);
 
+/* Producer side: fold the block rotation into a dense weight matrix and round
+ * it to ternary g128 (openbonsai.org, "How it works", steps 1 "Rotate" and
+ * 2 "Round"; the pages round with sequential GPTQ on calibration data, which
+ * needs a model and data; this is the plain stand-in).
+ *   w      : device [N, K] row-major, wt in {BF16, FP16, FP32}, 4-byte aligned.
+ *   signs  : device K int8 (+-1) of the layer's rotation, 8-byte aligned; NULL
+ *            = w is already folded (only rounded).
+ *   Fold   : w'_b = H (d_b * w_b) / 32 per row and 1024-block (W' = W R).
+ *   Round  : per 128-group s = fp16(mean |w'|) (nearest, ties to even),
+ *            t = clip(rint(w' / s), -1, 1) (rint: halves to even), t = 0 where
+ *            s = 0.
+ *   packed : device, tb_packed_bytes(f, N, K) bytes, 16-byte aligned (2-bit
+ *            slots or base-3); scales: device [N, K/128] fp16 bits.  Both
+ *            written in full, nothing else touched.
+ * Computed in fp64 with one rounding to fp16 for the scale: wherever the fp64
+ * sums of the fold and of the group's |w'| are exact (all bf16 and fp16 input;
+ * fp32 input spanning fewer than about 40 binary orders inside a block) the
+ * codes and scales equal those of exact arithmetic.  K % 1024 == 0 (else
+ * TB_ERR_SHAPE); TB_FMT_2BIT or TB_FMT_BASE3 (else TB_ERR_FORMAT). */
+tb_status tb_prepare_weights(const void* w, tb_dtype wt, const int8_t* signs, int64_t N, int64_t K,
+                             tb_format f, uint8_t* packed, uint16_t* scales, void* stream);
+
 /* Device workspace bytes tb_ternary_linear needs for these sizes (any path,
  * any dtype).  0 means none.  Returns 0 also for invalid sizes. */
 size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K);
@@ -211,10 +233,13 @@ int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64
  *   Takes the arguments of tb_ternary_linear minus the workspace, with the
  *   GEMV path's rules: float mode, TB_FMT_2BIT, M <= 4, K % 1024 == 0, all
  *   pointers 16-byte aligned (else TB_ERR_SHAPE / TB_ERR_ALIGN / TB_ERR_DTYPE).
- *   The decode path needs max(M * (2K + K/16), 16K + M * K/16) bytes of
- *   scratch, which must fit TB_NOALLOC_SCRATCH_BYTES (576 KiB: e.g. K <= 32768
- *   at any M <= 4); larger sizes return TB_ERR_WORKSPACE ("too big for the
- *   library's fixed scratch") and nothing is launched.
+ *   The decode path needs M * (2K + K/16 + 8448) bytes of scratch, and for
+ *   one token at least K/128 * 280 bytes (the one-token kernel's activation
+ *   words when K is too long for it to rotate x itself); the larger figure
+ *   must fit TB_NOALLOC_SCRATCH_BYTES (576 KiB), which allows K up to 269312
+ *   at M = 1, 138240 at M = 2, 91136 at M = 3 and 66560 at M = 4.  Larger
+ *   sizes return TB_ERR_WORKSPACE ("too big for the library's fixed
+ *   scratch") and nothing is launched.
  *   Every GPU that loads the library holds the scratch until the process exits.
  *   The first call on a device looks up the scratch's device address (a host
  *   call that does not allocate); make that first call before any stream

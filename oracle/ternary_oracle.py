@@ -23,7 +23,7 @@ What the layer computes (sources are the pages' sections):
   there only as "dense trit" and "2-bit slot" packings; the byte layouts below
   are this library's own definitions of those two ideas.
 
-Readings taken where the pages are silent (each is stated again in the design doc):
+Readings taken where the pages are silent:
 
 * R_b = diag(d_b) H / 32 with H the Sylvester Hadamard matrix of order 1024 in
   natural order and d_b the +-1 signs of block b; the run-time transform is

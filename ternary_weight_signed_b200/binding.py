@@ -31,6 +31,7 @@ _SIGNATURES = {
     "tb_pack_ternary": (_int, [_int, _vp, _i64, _i64, _vp, _vp, _vp]),
     "tb_unpack_ternary": (_int, [_int, _vp, _i64, _i64, _vp, _vp, _vp]),
     "tb_hadamard_rotate": (_int, [_vp, _int, _vp, _int, _vp, _i64, _i64, _int, _vp]),
+    "tb_prepare_weights": (_int, [_vp, _int, _vp, _i64, _i64, _int, _vp, _vp, _vp]),
     "tb_ternary_linear_workspace": (_sz, [_int, _i64, _i64, _i64]),
     "tb_ternary_linear": (_int, [_vp, _int, _vp, _vp, _int, _i64, _i64, _i64, _vp, _vp, _int,
                                  _vp, _sz, _vp]),
@@ -137,6 +138,12 @@ def tb_hadamard_rotate(x, xt, y, yt, signs, m, k, inverse=0, stream=None, check=
     st = load().tb_hadamard_rotate(_ptr(x), xt, _ptr(y), yt, _ptr(signs), m, k, int(inverse),
                                    _stream(stream))
     return _done(st, "tb_hadamard_rotate", check)
+
+
+def tb_prepare_weights(w, wt, signs, n, k, fmt, packed, scales, stream=None, check=True):
+    st = load().tb_prepare_weights(_ptr(w), wt, _ptr(signs), n, k, _fmt(fmt), _ptr(packed),
+                                   _ptr(scales), _stream(stream))
+    return _done(st, "tb_prepare_weights", check)
 
 
 def tb_ternary_linear_workspace(fmt, m, n, k) -> int:

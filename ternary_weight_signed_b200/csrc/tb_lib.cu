@@ -17,6 +17,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_m1.cuh"
+#include "prepare.cuh"
 #include "gemv_b3.cuh"
 #include "gemv_tc.cuh"
 #include "hadamard.cuh"
@@ -1065,6 +1066,39 @@ tb_status tb_hadamard_rotate(const void* x, tb_dtype xt, void* y, tb_dtype yt, c
   return launch_status();
 }
 
+tb_status tb_prepare_weights(const void* w, tb_dtype wt, const int8_t* signs, int64_t N, int64_t K, tb_format f,
+                             uint8_t* packed, uint16_t* scales, void* stream) {
+  if (f != TB_FMT_2BIT && f != TB_FMT_BASE3) return TB_ERR_FORMAT;
+  if (w == nullptr || packed == nullptr || scales == nullptr) return TB_ERR_NULL;
+  if (!is_float_dtype(wt)) return TB_ERR_DTYPE;
+  if (N < 1 || K < 1024 || K % 1024 != 0 || K > kMaxDim || K / 1024 > 65535 ||
+      (N + kPwWarps - 1) / kPwWarps > 65535)
+    return TB_ERR_SHAPE;
+  if (!aligned(w, 4) || !aligned(packed, 16) || !aligned(scales, 2) || (signs != nullptr && !aligned(signs, 8)))
+    return TB_ERR_ALIGN;
+  const DevInfo* d = nullptr;
+  const tb_status st = current_device(&d);
+  if (st != TB_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  const dim3 grid(static_cast<unsigned>(K / 1024), static_cast<unsigned>((N + kPwWarps - 1) / kPwWarps));
+  const dim3 block(32 * kPwWarps);
+  const int k = static_cast<int>(K);
+#define TB_PW(T)                                                                                                  \
+  do {                                                                                                          \
+    if (f == TB_FMT_2BIT)                                                                                       \
+      prepare_weights_kernel<T, 0><<<grid, block, 0, s>>>(static_cast<const T*>(w), signs, packed, scales, N, k); \
+    else                                                                                                        \
+      prepare_weights_kernel<T, 1><<<grid, block, 0, s>>>(static_cast<const T*>(w), signs, packed, scales, N, k); \
+  } while (0)
+  switch (wt) {
+    case TB_BF16: TB_PW(__nv_bfloat16); break;
+    case TB_FP16: TB_PW(__half); break;
+    default: TB_PW(float); break;
+  }
+#undef TB_PW
+  return launch_status();
+}
+
 size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K) {
   if ((f != TB_FMT_2BIT && f != TB_FMT_BASE3) || M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
   return workspace_bytes(M, K) + b3_transcode_bytes(f, M, N, K);
@@ -1108,6 +1142,16 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[TB_NOALLOC_SCRATCH_BY
 static std::mutex g_noalloc_mu;
 static void* g_noalloc_ptr[64] = {};
 
+// Scratch the decode path can write for M tokens of width K: the activation
+// stages of the CUDA-core decode (every M) and, for one token with K past the
+// fused-rotation limit, the prep kernel's output for the one-token kernel.
+// The larger of the two, whichever kernel the shape then selects.
+static int64_t noalloc_need(int64_t M, int64_t K) {
+  const int64_t v = gemv_ws_bytes(M, K);
+  const int64_t g1 = M == 1 ? g1_act_bytes(K) : 0;
+  return v > g1 ? v : g1;
+}
+
 static tb_status noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -1139,8 +1183,7 @@ tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* p
   if (st != TB_OK) return st;
   if (xt == TB_INT8) return TB_ERR_DTYPE;
   if (M > kGemvMaxM || K % 1024 != 0) return TB_ERR_SHAPE;
-  const int64_t need = gemv_ws_bytes(M, K);
-  if (need > static_cast<int64_t>(TB_NOALLOC_SCRATCH_BYTES)) return TB_ERR_WORKSPACE;
+  if (noalloc_need(M, K) > static_cast<int64_t>(TB_NOALLOC_SCRATCH_BYTES)) return TB_ERR_WORKSPACE;
   if (!aligned(packed, 16) || !aligned(scales, 16) || !aligned(x, 16) || !aligned(y, 16) ||
       (signs != nullptr && !aligned(signs, 16)))
     return TB_ERR_ALIGN;

@@ -145,3 +145,48 @@ def test_fault_query_needs_pointer(lib):
 def test_ctypes_signatures_are_set(lib):
     assert lib.tb_ternary_linear.restype is ctypes.c_int
     assert len(lib.tb_ternary_linear_ex.argtypes) == 15
+
+
+def _noalloc_need(m, k):
+    """Scratch the decode path may write for m tokens of width k: the CUDA-core
+    decode's activation stages, and for one token the one-token kernel's
+    activation words (280 bytes per 128-group)."""
+    need = m * (2 * k + k // 16 + 8448)
+    if m == 1:
+        need = max(need, (k // 128) * 280)
+    return need
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4])
+def test_noalloc_size_check_covers_every_decode_path(lib, m):
+    # An accepted size passes the scratch check and then stops at the
+    # alignment check (y is 4- but not 16-byte aligned), so nothing reaches the
+    # device; a rejected one returns TB_ERR_WORKSPACE.  The boundary must be
+    # where the scratch of every kernel the decode path can pick still fits.
+    limit = tb.TB_NOALLOC_SCRATCH_BYTES
+    largest = 0
+    for blocks in range(1, 300):
+        k = 1024 * blocks
+        st = tb.tb_ternary_linear_noalloc(FAKE, tb.TB_BF16, FAKE, FAKE, m, 256, k, FAKE, FAKE + 4,
+                                          tb.TB_FP32, stream=0, check=False)
+        fits = _noalloc_need(m, k) <= limit
+        assert st == (tb.TB_ERR_ALIGN if fits else tb.TB_ERR_WORKSPACE), (m, k, st)
+        if fits:
+            largest = k
+            assert (k // 128) * 280 <= limit or m > 1
+    assert largest == {1: 269312, 2: 138240, 3: 91136, 4: 66560}[m]
+
+
+def test_prepare_validation(lib):
+    f = tb.tb_prepare_weights
+    bf = tb.TB_BF16
+    assert f(FAKE, bf, FAKE, 4, 1024, 9, FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_FORMAT
+    assert f(None, bf, FAKE, 4, 1024, "2bit", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_NULL
+    assert f(FAKE, bf, FAKE, 4, 1024, "2bit", None, FAKE, stream=0, check=False) == tb.TB_ERR_NULL
+    assert f(FAKE, bf, FAKE, 4, 1024, "2bit", FAKE, None, stream=0, check=False) == tb.TB_ERR_NULL
+    assert f(FAKE, tb.TB_INT8, FAKE, 4, 1024, "2bit", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_DTYPE
+    assert f(FAKE, bf, FAKE, 4, 1536, "2bit", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_SHAPE
+    assert f(FAKE, bf, FAKE, 0, 1024, "base3", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_SHAPE
+    assert f(FAKE + 2, bf, FAKE, 4, 1024, "2bit", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_ALIGN
+    assert f(FAKE, bf, FAKE, 4, 1024, "2bit", FAKE + 8, FAKE, stream=0, check=False) == tb.TB_ERR_ALIGN
+    assert f(FAKE, bf, FAKE + 4, 4, 1024, "2bit", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_ALIGN

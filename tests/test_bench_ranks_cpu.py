@@ -30,9 +30,10 @@ def _worker(rank, world, port, outdir):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         bench._barrier(world)
-        # rank r "took" 1 + r ms per step
+        # rank r "took" 1 + r ms per call
         ms = bench._max_over_ranks(1.0 + rank, torch.device("cpu"), world)
-        res = {"step_bytes": 10 ** 9, "ms_per_step": ms, "steps": 10, "path": 1, "copies": 2}
+        res = {"step_bytes": 10 ** 9, "ms_per_call": ms, "ms_per_step": 1000 * ms, "calls_per_step": 1000,
+               "per_call_spread": {}, "steps": 10, "path": 1, "copies": 2}
         entry = bench._decode_entry(res, 1000.0, "measured", world)
         with open(os.path.join(outdir, f"{rank}.json"), "w") as f:
             json.dump({"ms": ms, "value": entry["value"], "achieved": entry["roofline"]["achieved"],
@@ -48,7 +49,7 @@ def test_two_ranks_take_the_slowest_time(tmp_path):
     got = [json.load(open(tmp_path / f"{r}.json")) for r in range(world)]
     for g in got:
         assert g["ms"] == 2.0  # the slower rank's time, on every rank
-        # 1 GB per step in 2 ms = 500 GB/s per GPU; the job moves twice that
+        # 1 GB per call in 2 ms = 500 GB/s per GPU; the job moves twice that
         assert g["achieved"] == 500.0
         assert g["value"] == 1000.0
         assert g["frac"] == 0.5
