@@ -162,7 +162,7 @@ def _launches_per_call(tb, fmt, m, n, k):
     one-token 2-bit decode kernel rotates x itself up to K = 8192 (one launch);
     the other float paths run an activation prep kernel and one main kernel."""
     path = tb.tb_ternary_linear_path(tb.TB_BF16, fmt, m, n, k, True, True)
-    if path == tb.TB_PATH_GEMV and fmt == "2bit" and m == 1 and k // 1024 <= 8:
+    if path == tb.TB_PATH_GEMV and fmt in ("2bit", "1bit") and m == 1 and k // 1024 <= 8:
         return 1
     if path == tb.TB_PATH_GEMV and fmt == "base3":
         return 2 * ((m + 3) // 4)
@@ -353,11 +353,12 @@ def run_ours(args, rank, world):
     m, n, k = 1, w["n"], w["k"]
     stream = torch.cuda.Stream(device=dev)
     peak, peak_kind = _peaks()
-    fmts = [args.fmt] + [f for f in ("2bit", "base3") if f != args.fmt]
+    fmts = [args.fmt] + [f for f in ("2bit", "base3", "1bit") if f != args.fmt]
     main = None
     others = {}
     for fmt in fmts:
-        res = measure_decode(args, tb, inputs, dev, stream, fmt, m, n, k, w["seed"] + rank, w["p0"],
+        p0 = 0.0 if fmt == "1bit" else w["p0"]  # 1-bit codes are -1 or +1
+        res = measure_decode(args, tb, inputs, dev, stream, fmt, m, n, k, w["seed"] + rank, p0,
                              w["scale_kind"], w["outlier_rate"], world, sample=(fmt == args.fmt))
         if fmt == args.fmt:
             main = res
@@ -372,8 +373,9 @@ def run_ours(args, rank, world):
     head = _decode_entry(main, peak, peak_kind, world)
     roof = head["roofline"]
     roof["traffic"] = _traffic(args.fmt)
-    roof["kernel"] = ("tb_ternary_linear decode call (gemv1_2bit_kernel, rotation fused)" if args.fmt == "2bit"
-                      else "tb_ternary_linear decode call (prep_b3_kernel + gemv_b3_kernel)")
+    roof["kernel"] = {"2bit": "tb_ternary_linear decode call (gemv1_kernel, 2-bit, rotation fused)",
+                      "1bit": "tb_ternary_linear decode call (gemv1_kernel, 1-bit, rotation fused)",
+                      "base3": "tb_ternary_linear decode call (prep_b3_kernel + gemv_b3_kernel)"}[args.fmt]
     roof["timing"] = ("device time per call over the timed steps (back-to-back calls in a CUDA graph, CUDA events "
                       "on the launching stream)")
     return {
@@ -701,7 +703,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--fmt", default="2bit", choices=["2bit", "base3"])
+    ap.add_argument("--fmt", default="2bit", choices=["2bit", "base3", "1bit"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--sweep", action="store_true", help="print the down-projection decode sweep instead")

@@ -52,6 +52,14 @@
  *                  are the padding value 1).  Row stride 26*K/128 bytes.  A byte
  *                  >= 243, or a last byte whose digits 3, 4 are not both 1, is
  *                  invalid.  1.625 + 16/128 = 1.75 bits per weight.
+ *   TB_FMT_1BIT  : 1-bit g128, the pages' other shipped format (each weight
+ *                  -1 or +1 with one FP16 scale per 128; dev.to, "How Prism ML
+ *                  Squeezed a 27B Model Into 3.9 GB", "Two formats ship
+ *                  today").  Byte i of a row holds k = 8i..8i+7, weight 8i+j in
+ *                  bit j, bit 1 = +1 and bit 0 = -1.  Row stride K/8 bytes.
+ *                  Every byte is valid; the packer counts any code other than
+ *                  -1, +1 (0 included) and packs it as -1.  1 + 16/128 =
+ *                  1.125 bits per weight.
  *
  * Rotation (this library's reading of "signed block Hadamard"): for block b of
  * 1024 inputs with signs d_b in {-1,+1}, R_b = diag(d_b) H / 32 where H is the
@@ -83,6 +91,7 @@ typedef int tb_status;
 typedef int tb_format;
 #define TB_FMT_2BIT 0
 #define TB_FMT_BASE3 1
+#define TB_FMT_1BIT 2
 
 typedef int tb_dtype;
 #define TB_BF16 0
@@ -95,14 +104,16 @@ typedef int tb_path;
 #define TB_PATH_AUTO 0   /* choose by shape (what tb_ternary_linear does)       */
 #define TB_PATH_GEMV 1   /* CUDA-core streaming kernels on 16-bit fixed-point
                             activations, for M <= 4 (base-3: M <= 7, in chunks
-                            of 4 tokens).  One token (2-bit): one launch that
-                            rotates x itself for K <= 8192                     */
+                            of 4 tokens; 1-bit: M = 1).  One token (2-bit,
+                            1-bit): one launch that rotates x itself for
+                            K <= 8192                                          */
 #define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
                             s*t in shared memory, fp32 accumulators in TMEM);
                             base-3 from 8 tokens, re-encoded to 2-bit slots in
-                            the workspace first.  Chosen by TB_PATH_AUTO past
-                            16 tokens, or from 8 base-3 tokens when N is above
-                            the tensor-core decode's 148 * 128 rows            */
+                            the workspace first; 1-bit from 2 tokens.  Chosen
+                            by TB_PATH_AUTO past 16 tokens, or from 8 base-3
+                            tokens when N is above the tensor-core decode's
+                            148 * 128 rows                                    */
 #define TB_PATH_SIMPLE 3 /* plain per-row kernel: any K % 128, any alignment    */
 #define TB_PATH_GEMV_TC 4 /* tcgen05 decode kernel (codes unpacked into TMEM as
                             the u8 A operand, int8 activation planes as B in
@@ -126,7 +137,8 @@ size_t tb_packed_bytes(tb_format f, int64_t N, int64_t K);
  *   codes  : device, N*K int8.
  *   packed : device, tb_packed_bytes(f, N, K) bytes, written in full.
  *   d_invalid_count : device uint32 or NULL.  Every code outside {-1,0,1} is
- *            packed as 0 and, when non-NULL, adds 1 to *d_invalid_count.
+ *            packed as 0 (1-bit: every code outside {-1,+1} is packed as -1)
+ *            and, when non-NULL, adds 1 to *d_invalid_count.
  * Requires K % 128 == 0; codes and packed 16-byte aligned (else TB_ERR_ALIGN).
  * Defined by the format description above; no counterpart kernel on the pages. */
 tb_status tb_pack_ternary(tb_format f, const int8_t* codes, int64_t N, int64_t K,
@@ -134,7 +146,8 @@ tb_status tb_pack_ternary(tb_format f, const int8_t* codes, int64_t N, int64_t K
 
 /* Unpack format-f bytes into int8 codes [N, K].  Invalid slots/bytes decode to
  * 0 and, when d_invalid_count is non-NULL, add 1 each (2-bit: per slot holding
- * 3; base-3: per invalid byte).  Same size/alignment rules as tb_pack_ternary. */
+ * 3; base-3: per invalid byte; 1-bit has none).  Same size/alignment rules as
+ * tb_pack_ternary. */
 tb_status tb_unpack_ternary(tb_format f, const uint8_t* packed, int64_t N, int64_t K,
                             int8_t* codes, uint32_t* d_invalid_count, void* stream);
 

@@ -15,11 +15,11 @@ from . import build as _build
 
 TB_OK, TB_ERR_NULL, TB_ERR_SHAPE, TB_ERR_DTYPE, TB_ERR_FORMAT = 0, 1, 2, 3, 4
 TB_ERR_ALIGN, TB_ERR_CUDA, TB_ERR_WORKSPACE, TB_ERR_DEVICE = 5, 6, 7, 8
-TB_FMT_2BIT, TB_FMT_BASE3 = 0, 1
+TB_FMT_2BIT, TB_FMT_BASE3, TB_FMT_1BIT = 0, 1, 2
 TB_BF16, TB_FP16, TB_FP32, TB_INT8, TB_INT32 = 0, 1, 2, 3, 4
 TB_PATH_AUTO, TB_PATH_GEMV, TB_PATH_GEMM, TB_PATH_SIMPLE, TB_PATH_GEMV_TC = 0, 1, 2, 3, 4
 
-FORMATS = {"2bit": TB_FMT_2BIT, "base3": TB_FMT_BASE3}
+FORMATS = {"2bit": TB_FMT_2BIT, "base3": TB_FMT_BASE3, "1bit": TB_FMT_1BIT}
 
 HEADER = os.path.join(_build.ROOT, "include", "ternary_b200.h")
 

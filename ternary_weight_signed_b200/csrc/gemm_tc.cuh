@@ -1,5 +1,6 @@
 // Prefill GEMM on the 5th-generation tensor cores (tcgen05 + TMEM), 2-bit
-// slot format.
+// slot format (and 1-bit g128, unpacked the same way to exact fp16 s*t with
+// t = -1 or +1).
 //
 // y[m, n] = sum_k x'[m, k] * w[n, k],  w = s[n, k/128] * t[n, k]  (ternary
 // g128: news.ditty.ir, second paragraph).  Once unpacked the product is a dense
@@ -207,10 +208,14 @@ __device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, c
   }
 }
 
-template <int BM, int BN, typename TOut>
+// kFmt: 0 = 2-bit slots (16 bytes of a row per 64-code stage), 2 = 1-bit (16
+// bytes per 128 codes: the box of an even stage also carries the codes of the
+// odd stage after it, which the unpack threads keep in registers).
+template <int BM, int BN, typename TOut, int kFmt>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_2bit_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                        const GemmParams p) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                   const GemmParams p) {
+  static_assert(kFmt == 0 || kFmt == 2, "2-bit or 1-bit codes");
   static_assert(BN % 32 == 0 && BN >= 128 && BN <= kGemmBN, "weight tile width");
   static_assert(BM == 128 || BM == 256, "token tile");
   constexpr int kA = gemm_a_bytes(BM), kStage = gemm_stage_bytes(BM, BN), kB = gemm_b_bytes(BN),
@@ -259,9 +264,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             !mbar_wait(&empty[s], ((kb / kGemmStages) & 1) ^ 1, FAULT_WAIT_EMPTY))
           break;
         uint8_t* st = smem + s * kStage;
-        mbar_arrive_expect_tx(&full[s], kA + kW);
+        const bool wload = kFmt == 0 || (kb & 1) == 0;
+        mbar_arrive_expect_tx(&full[s], kA + (wload ? kW : 0));
         tma_load_2d(st, &tm_x, kb * kGemmBK, m0, &full[s]);
-        tma_load_2d(st + kA + kB, &tm_w, kb * (kGemmBK / 16), n0, &full[s]);
+        // x in 32-bit words: 2-bit, 4 words per stage; 1-bit, 4 words per two stages
+        if (wload) tma_load_2d(st + kA + kB, &tm_w, kFmt == 0 ? kb * 4 : (kb >> 1) * 4, n0, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -303,6 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const __half2 k1 = __float2half2_rn(1.f);
     const __half2 kinv256 = __float2half2_rn(1.f / 256.f);
     const __half2 km4 = __float2half2_rn(-4.f);
+    uint32_t wcur[2] = {0u, 0u}, wnext[2] = {0u, 0u};  // 1-bit codes of this and the next stage
     bool ok = true;
     for (int kb = 0; kb < nk && ok; ++kb) {
       const int s = kb % kGemmStages;
@@ -316,12 +324,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (g + 1 < G) s_next = __ushort_as_half(row_ok ? srow[g + 1] : uint16_t(0));
       }
       uint8_t* st = smem + s * kStage;
-      const uint4 w4 = in_tile ? *reinterpret_cast<const uint4*>(st + kA + kB + r * 16) : make_uint4(0, 0, 0, 0);
       const __half2 s2 = __halves2half2(s_cur, s_cur);
       const __half2 ns2 = __hneg2(s2);
       uint8_t* row = st + kA + r * 128;
+      if constexpr (kFmt == 2) {
+        // 1-bit: 16-code chunk c of the stage (c = 0..3) is half c & 1 of
+        // word c >> 1.  z holds its low 8 codes in bits 0-7 and its high 8 in
+        // bits 16-23; (z << (15 - j)) & 0x80008000 puts codes j and j + 8 on
+        // the sign bits of a half2, and XOR with (-s, -s) gives (s t_j, s t_{j+8}).
+        if ((kb & 1) == 0 && in_tile) {
+          const uint4 w4 = *reinterpret_cast<const uint4*>(st + kA + kB + r * 16);
+          wcur[0] = w4.x;
+          wcur[1] = w4.y;
+          wnext[0] = w4.z;
+          wnext[1] = w4.w;
+        } else if (in_tile) {
+          wcur[0] = wnext[0];
+          wcur[1] = wnext[1];
+        }
+        const uint32_t nb = *reinterpret_cast<const uint32_t*>(&ns2);
 #pragma unroll
-      for (int wd = 0; wd < 4 && in_tile; ++wd) {
+        for (int c = 0; c < 4 && in_tile; ++c) {
+          const uint32_t z = __byte_perm(wcur[c >> 1], 0u, (c & 1) ? 0x4342u : 0x4140u);
+          uint32_t o[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) o[j] = ((z << (15 - j)) & 0x80008000u) ^ nb;
+          *reinterpret_cast<uint4*>(row + 16 * ((2 * c) ^ sw)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(row + 16 * ((2 * c + 1) ^ sw)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+      const uint4 w4 = (kFmt == 0 && in_tile) ? *reinterpret_cast<const uint4*>(st + kA + kB + r * 16)
+                                              : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int wd = 0; wd < 4 && in_tile && kFmt == 0; ++wd) {
         const uint32_t w = (&w4.x)[wd];
         uint32_t o[8];
 #pragma unroll

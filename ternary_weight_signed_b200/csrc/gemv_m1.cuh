@@ -61,6 +61,13 @@
 
 namespace tb {
 
+// Packed formats this kernel reads (the library's format numbers): 2-bit slots
+// (128 bytes of a row per 512-code chunk, 128-byte swizzle) and 1-bit (64
+// bytes per chunk, 64-byte swizzle).
+constexpr int kG1Fmt2Bit = 0;
+constexpr int kG1Fmt1Bit = 2;
+__host__ __device__ constexpr uint32_t g1_box_bytes(int fmt) { return fmt == kG1Fmt1Bit ? 64u : 128u; }
+
 constexpr int kG1Warps = 8;
 constexpr int kG1Threads = 32 * kG1Warps;
 // Shared memory per CTA for two CTAs per SM (228 KB per SM, 1 KB reserved per CTA).
@@ -173,7 +180,7 @@ __device__ __forceinline__ void g1_fwht32(float (&v)[32]) {
 // row, so neither the 4-byte stores of a row nor the 16-byte loads of a
 // quarter-warp meet a bank twice); lane r then holds the 32 values of row r
 // and transforms over c.  Lane a ends with x'[32 a .. 32 a + 31].
-template <typename TIn>
+template <typename TIn, int kFmt>
 __device__ __forceinline__ bool g1_rotate_block(const TIn* __restrict__ x, const int8_t* sgn, uint64_t* sbar,
                                                 int blk, int G, uint8_t* act, float* xbuf, int lane) {
   const TIn* xb = x + static_cast<int64_t>(blk) * kHB;
@@ -241,19 +248,32 @@ __device__ __forceinline__ bool g1_rotate_block(const TIn* __restrict__ x, const
   int qs = static_cast<int>(qsb - 32u * 0x4B400000u);
   qs += __shfl_xor_sync(0xffffffffu, qs, 1);
   qs += __shfl_xor_sync(0xffffffffu, qs, 2);
-  // lane a holds codes 32 (a & 3) .. + 31 of group a >> 2, i.e. words
-  // i = 2 (a & 3) + i2 (i2 = 0, 1); word 8 i + 2 j + h pairs codes
-  // 16 i + 8 h + j and 16 i + 8 h + 4 + j
   uint32_t wv[16];
+  if constexpr (kFmt == kG1Fmt2Bit) {
+    // lane a holds codes 32 (a & 3) .. + 31 of group a >> 2, i.e. packed
+    // words i = 2 (a & 3) + i2 (i2 = 0, 1); word 8 i + 2 j + h pairs codes
+    // 16 i + 8 h + j and 16 i + 8 h + 4 + j
 #pragma unroll
-  for (int i2 = 0; i2 < 2; ++i2)
+    for (int i2 = 0; i2 < 2; ++i2)
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int u = 16 * i2 + 8 * h + j;
+          wv[8 * i2 + 2 * j + h] = __byte_perm(qb[u], qb[u + 4], 0x5410);
+        }
+  } else {
+    // 1-bit: lane a holds the 32 codes of packed word i = a & 3 of group
+    // a >> 2; word 16 i + 2 j + h pairs codes 32 i + 16 h + j and
+    // 32 i + 16 h + 8 + j
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int u = 16 * i2 + 8 * h + j;
-        wv[8 * i2 + 2 * j + h] = __byte_perm(qb[u], qb[u + 4], 0x5410);
+        const int u = 16 * h + j;
+        wv[2 * j + h] = __byte_perm(qb[u], qb[u + 8], 0x5410);
       }
+  }
   const int g = blk * 8 + (lane >> 2);
   uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupStride + 64 * (lane & 3));
 #pragma unroll
@@ -272,7 +292,7 @@ __device__ __forceinline__ bool g1_rotate_block(const TIn* __restrict__ x, const
 // lane, bits 4-8 across lanes, bit 9 across the two warps through `xch` (1024
 // floats of the pair's own; named barrier `bar`, 64 threads).  Then each
 // lane's 16 codes are word (l & 7) of group 8 blk + 4 hf + l / 8.
-template <typename TIn>
+template <typename TIn, int kFmt>
 __device__ __forceinline__ void g1_rotate_half(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
                                                int blk, int hf, int G, uint8_t* act, float* xch, int bar, int lane) {
   const int64_t e0 = static_cast<int64_t>(blk) * kHB + 512 * hf + 16 * lane;
@@ -339,16 +359,28 @@ __device__ __forceinline__ void g1_rotate_half(const TIn* __restrict__ x, const 
   }
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
-  uint32_t wv[8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      wv[2 * j + h] = __byte_perm(static_cast<uint32_t>(q[8 * h + j]), static_cast<uint32_t>(q[8 * h + j + 4]), 0x5410);
   const int g = blk * 8 + 4 * hf + (lane >> 3);
-  uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupStride + 32 * (lane & 7));
-  dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-  dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+  if constexpr (kFmt == kG1Fmt2Bit) {
+    // the lane's 16 codes are packed word l & 7 of the group
+    uint32_t wv[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        wv[2 * j + h] =
+            __byte_perm(static_cast<uint32_t>(q[8 * h + j]), static_cast<uint32_t>(q[8 * h + j + 4]), 0x5410);
+    uint4* dst = reinterpret_cast<uint4*>(act + g * kG1GroupStride + 32 * (lane & 7));
+    dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+  } else {
+    // 1-bit: the lane's 16 codes are half hh = l & 1 of packed word
+    // i = (l & 7) / 2, i.e. the words 16 i + 2 j + hh (j = 0..7)
+    const int i = (lane & 7) >> 1, hh = lane & 1;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(act + g * kG1GroupStride) + 16 * i + hh;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      dst[2 * j] = __byte_perm(static_cast<uint32_t>(q[j]), static_cast<uint32_t>(q[j + 8]), 0x5410);
+  }
   if ((lane & 7) == 0) {
     int2 inf;
     inf.x = __float_as_int(e);
@@ -361,7 +393,7 @@ __device__ __forceinline__ void g1_rotate_half(const TIn* __restrict__ x, const 
 // written to `ws` in the layout above.  Waits for the previous kernel on the
 // stream (which may have produced x, or may still read ws) before touching
 // either.
-template <typename TIn>
+template <typename TIn, int kFmt>
 __global__ void __launch_bounds__(128) prep_gemv1_kernel(const TIn* __restrict__ x, const int8_t* __restrict__ signs,
                                                          uint8_t* __restrict__ ws, int K) {
   __shared__ __align__(16) float xbuf[4][512];
@@ -371,20 +403,23 @@ __global__ void __launch_bounds__(128) prep_gemv1_kernel(const TIn* __restrict__
   const bool live = blk < (K >> 10);
   pdl_wait();
   if (live)
-    g1_rotate_block<TIn>(x, signs != nullptr ? signs + static_cast<int64_t>(blk) * kHB : nullptr, nullptr, blk,
-                         K >> 7, ws, xbuf[threadIdx.x >> 5], lane);
+    g1_rotate_block<TIn, kFmt>(x, signs != nullptr ? signs + static_cast<int64_t>(blk) * kHB : nullptr, nullptr,
+                               blk, K >> 7, ws, xbuf[threadIdx.x >> 5], lane);
 }
 
 // ---------------------------------------------------------------- decode
 // Stage s: its chunks' weight boxes into slot `slot`, completing on `bar`.
+template <int kFmt>
 __device__ __forceinline__ void gemv1_issue(const CUtensorMap* tm, const Gemv1Params& p, uint8_t* ring,
                                             uint64_t* bar, int s, int slot, int r0) {
+  constexpr uint32_t kBox = g1_box_bytes(kFmt);
   const int C = p.K >> 9;
   const int nb = min(p.NB, C - s * p.NB);
   uint8_t* dst = ring + static_cast<int64_t>(slot) * p.slot_bytes;
-  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb) * static_cast<uint32_t>(p.R) * 128u);
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb) * static_cast<uint32_t>(p.R) * kBox);
   const uint64_t pol = l2_policy_evict_first();  // weights are read once per call
-  for (int b = 0; b < nb; ++b) tma_load_2d_hint(dst + b * p.box_stride, tm, (s * p.NB + b) * 128, r0, bar, pol);
+  for (int b = 0; b < nb; ++b)
+    tma_load_2d_hint(dst + b * p.box_stride, tm, (s * p.NB + b) * static_cast<int>(kBox), r0, bar, pol);
 }
 
 // sum_k c_k q_k of one row's group: 8 packed words against the group's 64
@@ -408,10 +443,43 @@ __device__ __forceinline__ int g1_group_dot(const uint4& wa, const uint4& wb, co
          ((t[0][3] + t[1][3]) >> 6);
 }
 
+// 1-bit: sum_k (t_k + 1) q_k = 2 sum_k b_k q_k of one row's group, b the bit
+// of code k: 4 packed words of 32 codes against the group's 64 activation
+// words.  Masking a word with 0x01010101 << j leaves bit j of each byte, i.e.
+// 2^j b of codes 8 c + j (c = 0..3), so dp2a.lo / dp2a.hi pair bytes 0, 1 /
+// 2, 3 with the words 16 i + 2 j + h; T_j is exact in int32 and
+// 2 sum b q = sum_j T_j / 2^(j - 1).  |T_j| <= 8 * 2 * 128 * 32512 < 2^31.
+__device__ __forceinline__ int g1_group_dot_1bit(const uint4& w4, const uint32_t (&A)[64]) {
+  const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+  int t[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t c = w[i] & (0x01010101u << j);
+      t[j] = dp2a_lo(A[16 * i + 2 * j], c, t[j]);
+      t[j] = dp2a_hi(A[16 * i + 2 * j + 1], c, t[j]);
+    }
+  }
+  return (t[0] << 1) + t[1] + (t[2] >> 1) + (t[3] >> 2) + (t[4] >> 3) + (t[5] >> 4) + (t[6] >> 5) + (t[7] >> 6);
+}
+
+// sum_k (t_k + 1) q_k of one row's group from the lane's piece of the box.
+template <int kFmt>
+__device__ __forceinline__ int g1_dot(const uint8_t* box, int pa, const uint32_t (&A)[64]) {
+  if constexpr (kFmt == kG1Fmt2Bit) {
+    const uint4 w0 = *reinterpret_cast<const uint4*>(box + pa);
+    const uint4 w1 = *reinterpret_cast<const uint4*>(box + (pa ^ 16));
+    return g1_group_dot(w0, w1, A);
+  } else {
+    return g1_group_dot_1bit(*reinterpret_cast<const uint4*>(box + pa), A);
+  }
+}
+
 // TPW: row tiles per warp at most (1, 2 or 4).
-template <typename TIn, typename TOut, bool kFused, int TPW>
+template <typename TIn, typename TOut, bool kFused, int TPW, int kFmt>
 __global__ void __launch_bounds__(kG1Threads, 2)
-    gemv1_2bit_kernel(const __grid_constant__ CUtensorMap tm_w, const Gemv1Params p) {
+    gemv1_kernel(const __grid_constant__ CUtensorMap tm_w, const Gemv1Params p) {
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -460,7 +528,8 @@ __global__ void __launch_bounds__(kG1Threads, 2)
         for (int b = 0; b < (p.K >> 10); ++b)
           bulk_load(act + b * 8 * kG1GroupStride, p.signs + static_cast<int64_t>(b) * kHB, kHB, pre_bar);
     }
-    for (int s = kG1Warps - 1 - warp; s < pre; s += kG1Warps) gemv1_issue(&tm_w, p, ring, &full[s], s, s, r0);
+    for (int s = kG1Warps - 1 - warp; s < pre; s += kG1Warps)
+      gemv1_issue<kFmt>(&tm_w, p, ring, &full[s], s, s, r0);
     if constexpr (!kFused) {
       if (warp == kG1Warps - 1) {
         pdl_wait();  // the prep kernel's activation words
@@ -474,7 +543,8 @@ __global__ void __launch_bounds__(kG1Threads, 2)
     if (g1_half_blocks(p.K)) {
       pdl_wait();  // x may be the previous kernel's output
       if (warp < 2 * nblk)
-        g1_rotate_half<TIn>(x, p.signs, warp >> 1, warp & 1, G, act, red + (warp >> 1) * kHB, 1 + (warp >> 1), lane);
+        g1_rotate_half<TIn, kFmt>(x, p.signs, warp >> 1, warp & 1, G, act, red + (warp >> 1) * kHB, 1 + (warp >> 1),
+                                  lane);
     } else {
       // block `warp` (K <= kG1FusedMaxBlocks blocks); its signs were staged
       // in shared memory before the wait
@@ -483,8 +553,9 @@ __global__ void __launch_bounds__(kG1Threads, 2)
       // the transpose buffer is this block's own slice of the activation words
       // (8 x 272 bytes, written only after the transpose)
       uint8_t* slice = act + warp * 8 * kG1GroupStride;
-      if (live && !g1_rotate_block<TIn>(x, p.signs != nullptr ? reinterpret_cast<const int8_t*>(slice) : nullptr,
-                                        pre_bar, warp, G, act, reinterpret_cast<float*>(slice), lane) &&
+      if (live &&
+          !g1_rotate_block<TIn, kFmt>(x, p.signs != nullptr ? reinterpret_cast<const int8_t*>(slice) : nullptr,
+                                      pre_bar, warp, G, act, reinterpret_cast<float*>(slice), lane) &&
           lane == 0)
         atomicExch(cta_fault, 1u);
     }
@@ -496,17 +567,21 @@ __global__ void __launch_bounds__(kG1Threads, 2)
   const bool active = tg < p.Wt;
   const int t0 = tg * p.RT / p.Wt, nt = active ? (tg + 1) * p.RT / p.Wt - t0 : 0;  // this warp's row tiles
   const int2* info = reinterpret_cast<const int2*>(act + G * kG1GroupStride);
-  // byte offsets in a box of the lane's two 16-byte pieces (2 gslot and
-  // 2 gslot + 1 of the row's 128 bytes, swizzled with the row index mod 8 =
-  // rsub) and of the rows' scales; rows past the CTA's end read valid rows
-  // and their sums are dropped
-  const int u0 = ((2 * gslot) ^ rsub) << 4;
+  // byte offsets in a box of the lane's 16-byte pieces and of the rows'
+  // scales.  2-bit: pieces 2 gslot and 2 gslot + 1 of the row's 128 bytes,
+  // 128-byte swizzle (piece index XOR row mod 8 = rsub).  1-bit: piece gslot
+  // of the row's 64 bytes, 64-byte swizzle (piece index XOR (row / 2) mod 4 =
+  // rsub / 2).  Either way the eight rows of a quarter-warp land in eight
+  // different 16-byte bank groups.  Rows past the CTA's end read valid rows
+  // and their sums are dropped.
+  constexpr int kBox = static_cast<int>(g1_box_bytes(kFmt));
+  const int u0 = kFmt == kG1Fmt2Bit ? ((2 * gslot) ^ rsub) << 4 : (gslot ^ (rsub >> 1)) << 4;
   int pa[TPW], soff[TPW];
   float acc[TPW];
 #pragma unroll
   for (int i = 0; i < TPW; ++i) {
     const int r = 8 * (t0 + i) + rsub;
-    pa[i] = min(r, p.R - 1) * 128 + u0;
+    pa[i] = min(r, p.R - 1) * kBox + u0;
     soff[i] = min(r, nrows - 1) * G;
     acc[i] = 0.f;
   }
@@ -539,22 +614,16 @@ __global__ void __launch_bounds__(kG1Threads, 2)
     const int2 inf = info[g];
     const float e = __int_as_float(inf.x);
     if constexpr (TPW == 1) {
-      const uint4 w0 = *reinterpret_cast<const uint4*>(box + pa[0]);
-      const uint4 w1 = *reinterpret_cast<const uint4*>(box + (pa[0] ^ 16));
       const float sa = __half2float(sc[soff[0] + g]) * e;
-      acc[0] = fmaf(__int2float_rn(g1_group_dot(w0, w1, A) - inf.y), sa, acc[0]);
+      acc[0] = fmaf(__int2float_rn(g1_dot<kFmt>(box, pa[0], A) - inf.y), sa, acc[0]);
     } else {
 #pragma unroll
       for (int tp = 0; tp < TPW; tp += 2) {
         // tiles beyond nt compute on valid rows and are dropped at the end
-        const uint4 wa0 = *reinterpret_cast<const uint4*>(box + pa[tp]);
-        const uint4 wa1 = *reinterpret_cast<const uint4*>(box + (pa[tp] ^ 16));
-        const uint4 wb0 = *reinterpret_cast<const uint4*>(box + pa[tp + 1]);
-        const uint4 wb1 = *reinterpret_cast<const uint4*>(box + (pa[tp + 1] ^ 16));
         const float sa = __half2float(sc[soff[tp] + g]) * e;
         const float sb = __half2float(sc[soff[tp + 1] + g]) * e;
-        const int da = g1_group_dot(wa0, wa1, A) - inf.y;
-        const int db = g1_group_dot(wb0, wb1, A) - inf.y;
+        const int da = g1_dot<kFmt>(box, pa[tp], A) - inf.y;
+        const int db = g1_dot<kFmt>(box, pa[tp + 1], A) - inf.y;
         acc[tp] = fmaf(__int2float_rn(da), sa, acc[tp]);
         acc[tp + 1] = fmaf(__int2float_rn(db), sb, acc[tp + 1]);
       }
@@ -569,7 +638,7 @@ __global__ void __launch_bounds__(kG1Threads, 2)
         if (atomicAdd(&done[s], 1u) == static_cast<uint32_t>(nch * p.Wt - 1) && s + p.nslots < p.nstage) {
           __threadfence_block();
           issued[s + p.nslots] = 1u;
-          gemv1_issue(&tm_w, p, ring, &full[s + p.nslots], s + p.nslots, s % p.nslots, r0);
+          gemv1_issue<kFmt>(&tm_w, p, ring, &full[s + p.nslots], s + p.nslots, s % p.nslots, r0);
         }
       }
     }

@@ -1,4 +1,4 @@
-// Pack / unpack kernels for the two packed formats (byte layouts in
+// Pack / unpack kernels for the packed formats (byte layouts in
 // include/ternary_b200.h).  Elementwise, memory-bound, one thread per output
 // word (2-bit) or per 128-group (base-3).  Bit-exact by construction; invalid
 // input is counted, never trapped.
@@ -127,6 +127,48 @@ __global__ void unpack_base3_kernel(const uint16_t* __restrict__ in, int4* __res
     }
   }
   count_invalid(bad, counter);
+}
+
+// 1-bit g128 (each weight -1 or +1; dev.to, "How Prism ML Squeezed a 27B
+// Model Into 3.9 GB", the two formats that ship): weight k of a row in bit
+// k % 8 of byte k / 8, bit 1 = +1.  One thread per 32 codes -> one 32-bit word
+// (code u of the word in bit u).  Any code other than -1 and +1 (0 included)
+// is packed as -1 and counted.
+__global__ void pack_1bit_kernel(const int4* __restrict__ codes, uint32_t* __restrict__ out, int64_t nwords,
+                                 uint32_t* counter) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint32_t bad = 0;
+  if (i < nwords) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int4 v = codes[2 * i + h];
+      const int8_t* c = reinterpret_cast<const int8_t*>(&v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        bad += (c[j] != 1 && c[j] != -1) ? 1u : 0u;
+        w |= (c[j] == 1 ? 1u : 0u) << (16 * h + j);
+      }
+    }
+    out[i] = w;
+  }
+  count_invalid(bad, counter);
+}
+
+// Every bit pattern is valid: bit 1 -> +1, bit 0 -> -1.
+__global__ void unpack_1bit_kernel(const uint32_t* __restrict__ in, int4* __restrict__ codes, int64_t nwords) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i < nwords) {
+    const uint32_t w = in[i];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      int4 v;
+      int8_t* c = reinterpret_cast<int8_t*>(&v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) c[j] = ((w >> (16 * h + j)) & 1u) ? int8_t(1) : int8_t(-1);
+      codes[2 * i + h] = v;
+    }
+  }
 }
 
 // Base-3 groups (26 bytes) -> 2-bit slot groups (32 bytes): the 2-bit paths

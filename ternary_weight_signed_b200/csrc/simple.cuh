@@ -1,7 +1,7 @@
 // Plain per-row kernel for the ternary g128 product: one warp per output row,
 // lanes over 128-groups, codes decoded straight from the packed bytes with
-// byte loads.  It takes every shape and alignment the API allows (K % 128 == 0)
-// and both modes:
+// byte loads.  It takes every shape, alignment and packed format the API
+// allows (K % 128 == 0) and both modes:
 //   float  : y[m,n] = sum_g s[n,g] sum_{k in g} t[n,k] x'[m,k]   (x' fp32)
 //   integer: y[m,n] = sum_k t[n,k] x[m,k]                          (exact int32)
 // It is the path for shapes the fast kernels do not take, not a tuned kernel.
@@ -39,6 +39,16 @@ __device__ __forceinline__ int8_t group_code<1>(const uint8_t* __restrict__ grp,
   return invalid ? int8_t(0) : static_cast<int8_t>(static_cast<int>(dig[j]) - 1);
 }
 
+// 1-bit: bit k % 8 of byte k / 8, bit 1 = +1, bit 0 = -1.
+template <>
+__device__ __forceinline__ int8_t group_code<2>(const uint8_t* __restrict__ grp, int k) {
+  return ((grp[k >> 3] >> (k & 7)) & 1u) ? int8_t(1) : int8_t(-1);
+}
+
+// Packed bytes of one 128-group and of one row of K codes, per format
+// (0 = 2-bit slots, 1 = base-3, 2 = 1-bit).
+__host__ __device__ constexpr int simple_group_bytes(int fmt) { return fmt == 0 ? 32 : (fmt == 1 ? 26 : 16); }
+
 template <int FMT, bool INT_MODE, typename TX, typename TOut>
 __global__ void __launch_bounds__(32 * kSimpleWarps)
     simple_linear_kernel(const TX* __restrict__ x, const uint8_t* __restrict__ packed,
@@ -49,8 +59,8 @@ __global__ void __launch_bounds__(32 * kSimpleWarps)
   const int n = blockIdx.x * kSimpleWarps + warp;
   if (n >= N) return;
   const int G = K / 128;
-  const int64_t row_bytes = FMT == 0 ? K / 4 : static_cast<int64_t>(G) * 26;
-  const int grp_bytes = FMT == 0 ? 32 : 26;
+  constexpr int grp_bytes = simple_group_bytes(FMT);
+  const int64_t row_bytes = static_cast<int64_t>(G) * grp_bytes;
   const uint8_t* prow = packed + static_cast<int64_t>(n) * row_bytes;
   for (int m0 = 0; m0 < M; m0 += kSimpleMC) {
     const int mc = min(kSimpleMC, M - m0);

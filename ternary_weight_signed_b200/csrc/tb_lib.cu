@@ -288,8 +288,10 @@ struct G1Plan {
   Gemv1Layout lay;
 };
 
-// Geometry of the one-token decode kernel (gemv_m1.cuh); false if it does not fit.
-bool g1_plan(int64_t N, int64_t K, int sm_count, int max_smem, bool fused, G1Plan* out) {
+// Geometry of the one-token decode kernel (gemv_m1.cuh) for packed format
+// `fmt` (2-bit or 1-bit); false if it does not fit.
+bool g1_plan(int64_t N, int64_t K, int sm_count, int max_smem, bool fused, G1Plan* out, int fmt = TB_FMT_2BIT) {
+  const int64_t box = g1_box_bytes(fmt);
   if (K % 1024 != 0 || K < 1024 || N < 1 || sm_count < 1) return false;
   if (fused && K / kHB > kG1FusedMaxBlocks) return false;
   G1Plan pl;
@@ -318,9 +320,9 @@ bool g1_plan(int64_t N, int64_t K, int sm_count, int max_smem, bool fused, G1Pla
     }
   }
   if (best_cost < 0) return false;
-  pl.box_stride = static_cast<int>(align_up(R * 128, 1024));
+  pl.box_stride = static_cast<int>(align_up(R * box, 1024));
   // stages of at least 8 KB of weights, a power of two of chunks
-  int64_t want = (8192 + R * 128 - 1) / (R * 128);
+  int64_t want = (8192 + R * box - 1) / (R * box);
   if (want > C) want = C;
   int64_t nb = 1;
   pl.nb_log2 = 0;
@@ -455,10 +457,15 @@ constexpr int kB200SmemOptin = 232448;
 constexpr int kB3MaxM = kB3TranscodeMinM - 1;
 
 bool gemv_ok(const LinearArgs& a) {
-  const int64_t maxm = a.f == TB_FMT_BASE3 ? kB3MaxM : kGemvMaxM;
+  const int64_t maxm = a.f == TB_FMT_BASE3 ? kB3MaxM : (a.f == TB_FMT_1BIT ? 1 : kGemvMaxM);
   if (!(is_float_dtype(a.xt) && a.M >= 1 && a.M <= maxm && a.K % 1024 == 0 && fast_aligned(a) &&
         a.N < (int64_t(1) << 30)))
     return false;
+  if (a.f == TB_FMT_1BIT) {
+    // one token only, on the one-token kernel
+    G1Plan p1;
+    return g1_plan(a.N, a.K, kB200Sms, kB200SmemOptin, g1_fused(a.K), &p1, TB_FMT_1BIT);
+  }
   if (a.f == TB_FMT_BASE3) {
     B3Plan pl;
     return b3_plan(std::min<int64_t>(a.M, kGemvMaxM), a.N, a.K, kB200Sms, kB200SmemOptin, &pl);
@@ -491,6 +498,11 @@ bool gemm_ok(const LinearArgs& a) {
 
 int auto_path(const LinearArgs& a) {
   if (a.xt == TB_INT8) return TB_PATH_SIMPLE;
+  if (a.f == TB_FMT_1BIT) {
+    // 1-bit: the one-token decode, else the GEMM
+    if (gemv_ok(a)) return TB_PATH_GEMV;
+    return gemm_ok(a) ? TB_PATH_GEMM : TB_PATH_SIMPLE;
+  }
   // 2-bit: the dp4a kernel's cost grows with M, the tensor-core one's hardly
   // does; measured on B200 (K=17408, N=5120) the tensor-core kernel wins from
   // 4 tokens on (31 us against 40 us).
@@ -515,14 +527,14 @@ tb_status launch_gemv(const LinearArgs& a, const DevInfo* d, const GemvPlan& pl,
 
 // One token: gemv1_2bit_kernel, with the rotation inside it for K up to
 // kG1FusedMaxBlocks 1024-blocks, else after prep_gemv1_kernel.
-template <typename TIn, typename TOut, bool kFused>
+template <typename TIn, typename TOut, bool kFused, int kFmt>
 tb_status launch_gemv1(const LinearArgs& a, const DevInfo* d, const G1Plan& pl, const CUtensorMap& tm,
                        const Gemv1Params& p) {
   auto pick = [&]() {
     switch (pl.TPW) {
-      case 1: return gemv1_2bit_kernel<TIn, TOut, kFused, 1>;
-      case 2: return gemv1_2bit_kernel<TIn, TOut, kFused, 2>;
-      default: return gemv1_2bit_kernel<TIn, TOut, kFused, 4>;
+      case 1: return gemv1_kernel<TIn, TOut, kFused, 1, kFmt>;
+      case 2: return gemv1_kernel<TIn, TOut, kFused, 2, kFmt>;
+      default: return gemv1_kernel<TIn, TOut, kFused, 4, kFmt>;
     }
   };
   auto k = pick();
@@ -530,11 +542,14 @@ tb_status launch_gemv1(const LinearArgs& a, const DevInfo* d, const G1Plan& pl, 
   return launch_pdl(k, dim3(pl.grid), dim3(kG1Threads), static_cast<size_t>(pl.lay.bytes), a.st, tm, p);
 }
 
-template <typename TIn>
+template <typename TIn, int kFmt>
 tb_status run_gemv1_typed(const LinearArgs& a, const DevInfo* d, const G1Plan& pl) {
   CUtensorMap tm;
-  if (make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.packed, a.K / 4, a.N, a.K / 4, 128,
-                  static_cast<uint32_t>(pl.R), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+  // 2-bit: 128 bytes of a row per chunk, 128-byte swizzle; 1-bit: 64 bytes, 64-byte swizzle
+  const uint64_t row_bytes = kFmt == kG1Fmt1Bit ? a.K / 8 : a.K / 4;
+  if (make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.packed, row_bytes, a.N, row_bytes, g1_box_bytes(kFmt),
+                  static_cast<uint32_t>(pl.R),
+                  kFmt == kG1Fmt1Bit ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
   Gemv1Params p;
   p.x = pl.fused ? a.x : nullptr;
@@ -560,21 +575,28 @@ tb_status run_gemv1_typed(const LinearArgs& a, const DevInfo* d, const G1Plan& p
   p.off_bar = pl.lay.off_bar;
   if (!pl.fused) {
     const dim3 pgrid(static_cast<unsigned>((a.K / kHB + 3) / 4));
-    if (launch_pdl(prep_gemv1_kernel<TIn>, pgrid, dim3(128), 0, a.st, static_cast<const TIn*>(a.x), a.signs,
-                   static_cast<uint8_t*>(a.ws), static_cast<int>(a.K)) != TB_OK)
+    if (launch_pdl(prep_gemv1_kernel<TIn, kFmt>, pgrid, dim3(128), 0, a.st, static_cast<const TIn*>(a.x),
+                   a.signs, static_cast<uint8_t*>(a.ws), static_cast<int>(a.K)) != TB_OK)
       return TB_ERR_CUDA;
-    return a.yt == TB_FP32 ? launch_gemv1<TIn, float, false>(a, d, pl, tm, p)
-                           : launch_gemv1<TIn, __nv_bfloat16, false>(a, d, pl, tm, p);
+    return a.yt == TB_FP32 ? launch_gemv1<TIn, float, false, kFmt>(a, d, pl, tm, p)
+                           : launch_gemv1<TIn, __nv_bfloat16, false, kFmt>(a, d, pl, tm, p);
   }
-  return a.yt == TB_FP32 ? launch_gemv1<TIn, float, true>(a, d, pl, tm, p)
-                         : launch_gemv1<TIn, __nv_bfloat16, true>(a, d, pl, tm, p);
+  return a.yt == TB_FP32 ? launch_gemv1<TIn, float, true, kFmt>(a, d, pl, tm, p)
+                         : launch_gemv1<TIn, __nv_bfloat16, true, kFmt>(a, d, pl, tm, p);
 }
 
 template <typename TIn>
 tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
+  if (a.f == TB_FMT_1BIT) {
+    G1Plan p1;
+    if (a.M != 1 || !g1_plan(a.N, a.K, d->sm_count, d->max_smem_optin, g1_fused(a.K), &p1, TB_FMT_1BIT))
+      return TB_ERR_SHAPE;
+    return run_gemv1_typed<TIn, kG1Fmt1Bit>(a, d, p1);
+  }
   if (a.M == 1 && g1_preferred(a.N, a.K, d->sm_count)) {
     G1Plan p1;
-    if (g1_plan(a.N, a.K, d->sm_count, d->max_smem_optin, g1_fused(a.K), &p1)) return run_gemv1_typed<TIn>(a, d, p1);
+    if (g1_plan(a.N, a.K, d->sm_count, d->max_smem_optin, g1_fused(a.K), &p1))
+      return run_gemv1_typed<TIn, kG1Fmt2Bit>(a, d, p1);
   }
   GemvPlan pl;
   if (!gemv_plan(a.M, a.N, a.K, d->sm_count, d->max_smem_optin, &pl)) return TB_ERR_SHAPE;
@@ -826,7 +848,11 @@ tb_status run_simple_fmt(const LinearArgs& a) {
 }
 
 tb_status run_simple(const LinearArgs& a) {
-  return a.f == TB_FMT_2BIT ? run_simple_fmt<0>(a) : run_simple_fmt<1>(a);
+  switch (a.f) {
+    case TB_FMT_2BIT: return run_simple_fmt<0>(a);
+    case TB_FMT_BASE3: return run_simple_fmt<1>(a);
+    default: return run_simple_fmt<2>(a);
+  }
 }
 
 // ------------------------------------------------------------------ linear: tensor-core kernel
@@ -853,7 +879,9 @@ tb_status run_gemm(const LinearArgs& a, const DevInfo* d) {
   return run_gemm_2bit(c, d);
 }
 
+// 2-bit slots or 1-bit codes (base-3 arrives re-encoded to 2-bit slots).
 tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
+  const bool one_bit = a.f == TB_FMT_1BIT;
   __half* xh = static_cast<__half*>(a.ws);
   switch (a.xt) {
     case TB_BF16: launch_prep_gemm<__nv_bfloat16>(a, xh); break;
@@ -888,7 +916,9 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGemmBK,
                   static_cast<uint32_t>(bm), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
-  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, kGemmBK / 16,
+  // 16 bytes of a row per box: 64 codes (2-bit, one stage) or 128 codes (1-bit, two stages)
+  const uint64_t wrow = one_bit ? a.K / 8 : a.K / 4;
+  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, wrow / 4, a.N, wrow, 4,
                   static_cast<uint32_t>(bn)) != TB_OK)
     return TB_ERR_CUDA;
   GemmParams gp;
@@ -898,18 +928,23 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   gp.y = a.y;
   gp.scales = a.scales;
   const dim3 grid(static_cast<unsigned>((a.N + bn - 1) / bn), static_cast<unsigned>(mt));
-#define TB_GEMM_LAUNCH(BM, BN)                                                                             \
-  if (bm == BM && bn == BN) {                                                                              \
-    if (a.yt == TB_FP32) {                                                                                 \
-      auto k = gemm_2bit_tc_kernel<BM, BN, float>;                                                         \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                   \
+#define TB_GEMM_LAUNCH_F(BM, BN, F)                                                                         \
+  {                                                                                                          \
+    if (a.yt == TB_FP32) {                                                                                   \
+      auto k = gemm_tc_kernel<BM, BN, float, F>;                                                             \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
       return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BM, BN)), a.st, tm_x, \
-                        tm_w, gp);                                                                         \
-    }                                                                                                      \
-    auto k = gemm_2bit_tc_kernel<BM, BN, __nv_bfloat16>;                                                   \
-    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
+                        tm_w, gp);                                                                           \
+    }                                                                                                        \
+    auto k = gemm_tc_kernel<BM, BN, __nv_bfloat16, F>;                                                       \
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                       \
     return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BM, BN)), a.st, tm_x,   \
-                      tm_w, gp);                                                                           \
+                      tm_w, gp);                                                                             \
+  }
+#define TB_GEMM_LAUNCH(BM, BN)               \
+  if (bm == BM && bn == BN) {                \
+    if (one_bit) TB_GEMM_LAUNCH_F(BM, BN, 2) \
+    TB_GEMM_LAUNCH_F(BM, BN, 0)              \
   }
   TB_GEMM_LAUNCH(256, 256)
   TB_GEMM_LAUNCH(256, 192)
@@ -918,11 +953,14 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   TB_GEMM_LAUNCH(128, 192)
   TB_GEMM_LAUNCH(128, 128)
 #undef TB_GEMM_LAUNCH
+#undef TB_GEMM_LAUNCH_F
   return TB_ERR_SHAPE;
 }
 
+bool known_format(int f) { return f == TB_FMT_2BIT || f == TB_FMT_BASE3 || f == TB_FMT_1BIT; }
+
 tb_status validate_linear(const LinearArgs& a) {
-  if (a.f != TB_FMT_2BIT && a.f != TB_FMT_BASE3) return TB_ERR_FORMAT;
+  if (!known_format(a.f)) return TB_ERR_FORMAT;
   const bool int_mode = a.xt == TB_INT8;
   if (a.x == nullptr || a.packed == nullptr || a.y == nullptr) return TB_ERR_NULL;
   if (!int_mode && a.scales == nullptr) return TB_ERR_NULL;
@@ -996,12 +1034,13 @@ size_t tb_packed_bytes(tb_format f, int64_t N, int64_t K) {
   if (N <= 0 || K <= 0 || K % 128 != 0) return 0;
   if (f == TB_FMT_2BIT) return static_cast<size_t>(N) * static_cast<size_t>(K / 4);
   if (f == TB_FMT_BASE3) return static_cast<size_t>(N) * static_cast<size_t>(K / 128) * 26;
+  if (f == TB_FMT_1BIT) return static_cast<size_t>(N) * static_cast<size_t>(K / 8);
   return 0;
 }
 
 tb_status tb_pack_ternary(tb_format f, const int8_t* codes, int64_t N, int64_t K, uint8_t* packed,
                           uint32_t* d_invalid_count, void* stream) {
-  if (f != TB_FMT_2BIT && f != TB_FMT_BASE3) return TB_ERR_FORMAT;
+  if (!known_format(f)) return TB_ERR_FORMAT;
   if (codes == nullptr || packed == nullptr) return TB_ERR_NULL;
   if (N <= 0 || K <= 0 || K % 128 != 0 || N > kMaxDim || K > kMaxDim) return TB_ERR_SHAPE;
   if (!aligned(codes, 16) || !aligned(packed, 16) ||
@@ -1015,6 +1054,10 @@ tb_status tb_pack_ternary(tb_format f, const int8_t* codes, int64_t N, int64_t K
     const int64_t nw = N * K / 16;
     pack_2bit_kernel<<<static_cast<unsigned>((nw + 255) / 256), 256, 0, s>>>(
         reinterpret_cast<const int4*>(codes), reinterpret_cast<uint32_t*>(packed), nw, d_invalid_count);
+  } else if (f == TB_FMT_1BIT) {
+    const int64_t nw = N * K / 32;
+    pack_1bit_kernel<<<static_cast<unsigned>((nw + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const int4*>(codes), reinterpret_cast<uint32_t*>(packed), nw, d_invalid_count);
   } else {
     const int64_t ng = N * K / 128;
     pack_base3_kernel<<<static_cast<unsigned>((ng + 127) / 128), 128, 0, s>>>(
@@ -1025,7 +1068,7 @@ tb_status tb_pack_ternary(tb_format f, const int8_t* codes, int64_t N, int64_t K
 
 tb_status tb_unpack_ternary(tb_format f, const uint8_t* packed, int64_t N, int64_t K, int8_t* codes,
                             uint32_t* d_invalid_count, void* stream) {
-  if (f != TB_FMT_2BIT && f != TB_FMT_BASE3) return TB_ERR_FORMAT;
+  if (!known_format(f)) return TB_ERR_FORMAT;
   if (codes == nullptr || packed == nullptr) return TB_ERR_NULL;
   if (N <= 0 || K <= 0 || K % 128 != 0 || N > kMaxDim || K > kMaxDim) return TB_ERR_SHAPE;
   if (!aligned(codes, 16) || !aligned(packed, 16) ||
@@ -1039,6 +1082,10 @@ tb_status tb_unpack_ternary(tb_format f, const uint8_t* packed, int64_t N, int64
     const int64_t nw = N * K / 16;
     unpack_2bit_kernel<<<static_cast<unsigned>((nw + 255) / 256), 256, 0, s>>>(
         reinterpret_cast<const uint32_t*>(packed), reinterpret_cast<int4*>(codes), nw, d_invalid_count);
+  } else if (f == TB_FMT_1BIT) {
+    const int64_t nw = N * K / 32;
+    unpack_1bit_kernel<<<static_cast<unsigned>((nw + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const uint32_t*>(packed), reinterpret_cast<int4*>(codes), nw);
   } else {
     const int64_t ng = N * K / 128;
     unpack_base3_kernel<<<static_cast<unsigned>((ng + 127) / 128), 128, 0, s>>>(
@@ -1100,7 +1147,7 @@ tb_status tb_prepare_weights(const void* w, tb_dtype wt, const int8_t* signs, in
 }
 
 size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K) {
-  if ((f != TB_FMT_2BIT && f != TB_FMT_BASE3) || M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
+  if (!known_format(f) || M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
   return workspace_bytes(M, K) + b3_transcode_bytes(f, M, N, K);
 }
 

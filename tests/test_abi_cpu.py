@@ -92,6 +92,7 @@ def _lin(**kw):
 
 def test_linear_validation(lib):
     assert _lin(fmt=3) == tb.TB_ERR_FORMAT
+    assert _lin(fmt=-1) == tb.TB_ERR_FORMAT
     assert _lin(x=None) == tb.TB_ERR_NULL
     assert _lin(packed=None) == tb.TB_ERR_NULL
     assert _lin(scales=None) == tb.TB_ERR_NULL
@@ -190,3 +191,19 @@ def test_prepare_validation(lib):
     assert f(FAKE + 2, bf, FAKE, 4, 1024, "2bit", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_ALIGN
     assert f(FAKE, bf, FAKE, 4, 1024, "2bit", FAKE + 8, FAKE, stream=0, check=False) == tb.TB_ERR_ALIGN
     assert f(FAKE, bf, FAKE + 4, 4, 1024, "2bit", FAKE, FAKE, stream=0, check=False) == tb.TB_ERR_ALIGN
+
+
+@pytest.mark.parametrize("n,k", [(1, 128), (3, 384), (17408, 5120), (5120, 17408)])
+def test_packed_bytes_1bit(lib, n, k):
+    assert tb.tb_packed_bytes("1bit", n, k) == orc.packed_bytes("1bit", n, k) == n * k // 8
+
+
+def test_path_selection_1bit(lib):
+    p = tb.tb_ternary_linear_path
+    assert p(tb.TB_BF16, "1bit", 1, 17408, 5120) == tb.TB_PATH_GEMV
+    assert p(tb.TB_BF16, "1bit", 1, 5120, 17408) == tb.TB_PATH_GEMV
+    assert p(tb.TB_BF16, "1bit", 2, 17408, 5120) == tb.TB_PATH_GEMM
+    assert p(tb.TB_BF16, "1bit", 2048, 17408, 5120) == tb.TB_PATH_GEMM
+    assert p(tb.TB_BF16, "1bit", 1, 256, 640, has_signs=False) == tb.TB_PATH_SIMPLE
+    assert p(tb.TB_INT8, "1bit", 4, 256, 1024, has_signs=False) == tb.TB_PATH_SIMPLE
+    assert p(tb.TB_BF16, "1bit", 1, 17408, 5120, aligned16=False) == tb.TB_PATH_SIMPLE
