@@ -368,6 +368,7 @@ def run_ours(args, rank, world):
         res.pop("problem")
         torch.cuda.empty_cache()
     prefill = run_prefill(args, dev, stream, tb, inputs, world) if args.prefill else None
+    prefill_int = run_prefill(args, dev, stream, tb, inputs, world, integer=True) if args.prefill else None
     stack = (stack_cells(args, dev, stream, tb, inputs, ["2bit"], [1, 16], [0.33], ["separate", "shared_input"],
                          args.steps, inputs.STACK_LAYERS, world) if args.stack_leg else None)
     head = _decode_entry(main, peak, peak_kind, world)
@@ -403,19 +404,22 @@ def run_ours(args, rank, world):
         "formats": others,
         "e2e": e2e,
         "prefill": prefill,
+        "prefill_integer": prefill_int,
         "stack": stack,
         "gpu_launches": main["launches"],
         "clocks": main["clocks"],
     }
 
 
-def run_prefill(args, dev, stream, tb, inputs, world=1):
+def run_prefill(args, dev, stream, tb, inputs, world=1, integer=False):
     """Prefill GEMM workload (M=2048 tokens, K=5120, N=17408, 2-bit): tokens/s
     of the whole job (every rank one replica, timed as the slowest rank),
     TFLOP-equivalent/s per GPU (2*M*N*K per call) and its fraction of the
-    measured dense 16-bit tensor peak.  Successive calls take successive
-    copies of the weights (6) and of the activations (2), 185 MB together,
-    more than L2; the call is compute-bound."""
+    measured dense tensor peak.  Float mode: bf16 x rotated and rounded to
+    fp16, kind::f16 MMAs.  Integer mode (`integer`): int8 x, exact int32 y,
+    kind::i8 MMAs.  Successive calls take successive copies of the weights (6)
+    and of the activations (2), more than L2 together; the call is
+    compute-bound."""
     import torch
 
     w = inputs.WORKLOADS["prefill_m2048_k5120_n17408"]
@@ -429,16 +433,21 @@ def run_prefill(args, dev, stream, tb, inputs, world=1):
         tb.tb_pack_ternary("2bit", codes, n, k, pk)
     del codes
     scls = [torch.from_numpy(p.scales.view(np.int16)).to(dev) for _ in range(wcopies)]
-    xs = [torch.from_numpy(p.x_bf16.view(np.int16)).to(dev).view(torch.bfloat16) for _ in range(xcopies)]
-    signs = torch.from_numpy(p.signs).to(dev)
-    y = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+    if integer:
+        xi = np.random.default_rng(w["seed"]).integers(-127, 128, (m, k)).astype(np.int8)
+        xs = [torch.from_numpy(xi).to(dev) for _ in range(xcopies)]
+        xt, yt, ydt, signs = tb.TB_INT8, tb.TB_INT32, torch.int32, None
+    else:
+        xs = [torch.from_numpy(p.x_bf16.view(np.int16)).to(dev).view(torch.bfloat16) for _ in range(xcopies)]
+        xt, yt, ydt, signs = tb.TB_BF16, tb.TB_BF16, torch.bfloat16, torch.from_numpy(p.signs).to(dev)
+    y = torch.empty(m, n, dtype=ydt, device=dev)
     ws_bytes = tb.tb_ternary_linear_workspace("2bit", m, n, k)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     sh = stream.cuda_stream
 
     def call(i):
-        tb.tb_ternary_linear(xs[i % xcopies], tb.TB_BF16, packs[i % wcopies], scls[i % wcopies], "2bit", m, n, k,
-                             signs, y, tb.TB_BF16, ws, ws_bytes, stream=sh)
+        tb.tb_ternary_linear(xs[i % xcopies], xt, packs[i % wcopies], scls[i % wcopies], "2bit", m, n, k,
+                             signs, y, yt, ws, ws_bytes, stream=sh)
 
     calls = PREFILL_CALLS_PER_STEP
     with torch.cuda.stream(stream):
@@ -460,16 +469,20 @@ def run_prefill(args, dev, stream, tb, inputs, world=1):
     flops = 2.0 * m * n * k
     tflops = flops / (ms * 1e-3) / 1e12
     peak, kind = _tensor_peak()
-    return {"workload": "prefill GEMM M=2048 K=5120 N=17408 (2bit), bf16 in/out",
+    if integer:
+        peak, kind = 2.0 * peak, kind + " x 2 (nominal dense int8 : bf16 = 4.5 : 2.25 PFLOP/s)"
+    return {"workload": ("prefill GEMM M=2048 K=5120 N=17408 (2bit), " +
+                         ("int8 in, exact int32 out (integer mode)" if integer else "bf16 in/out")),
             "tok_s": round(m * world / (ms * 1e-3), 1), "ms_per_call": round(ms, 5),
             "calls_per_step": calls, "steps": args.steps, "ms_timed": round(total, 3),
-            "l2": "6 weight copies and 2 activation copies in rotation, 185 MB > 126 MB L2",
+            "l2": "6 weight copies and 2 activation copies in rotation, more than 126 MB L2",
             "per_call_spread": _spread(per, calls), "tflops_equiv": round(tflops, 2),
-            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
-                         "peak_source": kind, "dtype": "fp16 x fp16 -> fp32 (kind::f16)"},
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": round(peak, 1),
+                         "unit": "TFLOP/s" if not integer else "TOP/s", "frac": round(tflops / peak, 4),
+                         "peak_source": kind,
+                         "dtype": "s8 x u8 -> s32 (kind::i8)" if integer else "fp16 x fp16 -> fp32 (kind::f16)"},
             "clocks": clocks,
-            "kernel_path": tb.tb_ternary_linear_path(tb.TB_BF16, "2bit", m, n, k, True, True)}
+            "kernel_path": tb.tb_ternary_linear_path(xt, "2bit", m, n, k, not integer, True)}
 
 
 def _tensor_peak():

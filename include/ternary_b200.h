@@ -108,7 +108,11 @@ typedef int tb_path;
                             1-bit): one launch that rotates x itself for
                             K <= 8192                                          */
 #define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
-                            s*t in shared memory, fp32 accumulators in TMEM);
+                            s*t in shared memory, fp32 accumulators in TMEM;
+                            integer mode: kind::i8, int8 x times the biased
+                            codes, exact int32 accumulators, from 16 tokens,
+                            any K % 128, base-3 only with a workspace to
+                            re-encode into);
                             base-3 from 8 tokens, re-encoded to 2-bit slots in
                             the workspace first; 1-bit from 2 tokens.  Chosen
                             by TB_PATH_AUTO past 16 tokens, or from 8 base-3
@@ -199,6 +203,10 @@ size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K)
  *   scales  : device [N, K/128] fp16 bit patterns.  Ignored in integer mode.
  *   y       : device [M, N]; yt in {FP32, BF16} in float mode, INT32 in integer
  *             mode (y[m,n] = sum_k t[n,k] x[m,k], exact).
+ *   Integer mode needs no workspace (pass NULL, 0), except that base-3 weights
+ *   reach the tensor-core path (16 tokens and more) only when a workspace of
+ *   tb_ternary_linear_workspace bytes is passed to re-encode them into;
+ *   without one they take the plain kernel (same exact result).
  *   workspace : device, at least tb_ternary_linear_workspace(f, M, N, K) bytes,
  *             16-byte aligned; its contents on entry do not matter and are
  *             overwritten.  Must not be shared by calls in flight at once.

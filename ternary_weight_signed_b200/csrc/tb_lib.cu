@@ -15,6 +15,7 @@
 #include "tb_device.cuh"
 
 #include "gemm_tc.cuh"
+#include "gemm_i8.cuh"
 #include "gemv.cuh"
 #include "gemv_m1.cuh"
 #include "prepare.cuh"
@@ -496,8 +497,10 @@ bool gemm_ok(const LinearArgs& a) {
          (a.M + kGemmUM - 1) / kGemmUM <= 65535 && a.N < (int64_t(1) << 30);
 }
 
+bool gemm_i8_ok(const LinearArgs& a);
+
 int auto_path(const LinearArgs& a) {
-  if (a.xt == TB_INT8) return TB_PATH_SIMPLE;
+  if (a.xt == TB_INT8) return gemm_i8_ok(a) ? TB_PATH_GEMM : TB_PATH_SIMPLE;
   if (a.f == TB_FMT_1BIT) {
     // 1-bit: the one-token decode, else the GEMM
     if (gemv_ok(a)) return TB_PATH_GEMV;
@@ -879,6 +882,34 @@ tb_status run_gemm(const LinearArgs& a, const DevInfo* d) {
   return run_gemm_2bit(c, d);
 }
 
+// Tiles of the tensor-core GEMMs.  Token tile: 128 when it pads fewer token
+// rows than 256 (up to 128 tokens, and e.g. 300 tokens: 384 against 512 rows),
+// else 256, whose two MMAs share each unpacked weight tile.  Weight-tile
+// width: wave fill of the SMs times the tile's own efficiency.  Narrower tiles
+// reuse each activation stage for fewer weight rows and leave unpack warps
+// idle; on B200 the 192-wide tile ran the prefill shape (2048 x 17408 x 5120)
+// at 0.90 of the 256-wide tile's per-tile rate, which its better wave fill
+// (4.92 against 3.68 waves) does not make up.
+void gemm_tiles(int64_t M, int64_t N, int sm_count, int* bm_out, int* bn_out) {
+  const int bm = ((M + 127) / 128) * 128 < ((M + 255) / 256) * 256 ? 128 : 256;
+  const int64_t mt = (M + bm - 1) / bm;
+  int bn = 256;
+  double best = -1.0;
+  const int cands[3] = {256, 192, 128};
+  const double eff[3] = {1.0, 0.9, 0.8};
+  for (int i = 0; i < 3; ++i) {
+    const double tiles = static_cast<double>(((N + cands[i] - 1) / cands[i]) * mt);
+    const double waves = tiles / sm_count;
+    const double score = eff[i] * waves / std::ceil(waves);
+    if (score > best + 1e-9) {
+      best = score;
+      bn = cands[i];
+    }
+  }
+  *bm_out = bm;
+  *bn_out = bn;
+}
+
 // 2-bit slots or 1-bit codes (base-3 arrives re-encoded to 2-bit slots).
 tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   const bool one_bit = a.f == TB_FMT_1BIT;
@@ -889,29 +920,9 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
     default: launch_prep_gemm<float>(a, xh); break;
   }
   if (launch_status() != TB_OK) return TB_ERR_CUDA;
-  // Token tile: 128 when it pads fewer token rows than 256 (up to 128 tokens,
-  // and e.g. 300 tokens: 384 against 512 rows), else 256, whose two MMAs share
-  // each unpacked weight tile.
-  const int bm = ((a.M + 127) / 128) * 128 < ((a.M + 255) / 256) * 256 ? 128 : 256;
-  // Weight-tile width: wave fill of the SMs times the tile's own efficiency.
-  // Narrower tiles reuse each activation stage for fewer weight rows and leave
-  // unpack warps idle; on B200 the 192-wide tile ran the prefill shape
-  // (2048 x 17408 x 5120) at 0.90 of the 256-wide tile's per-tile rate, which
-  // its better wave fill (4.92 against 3.68 waves) does not make up.
+  int bm = 256, bn = 256;
+  gemm_tiles(a.M, a.N, d->sm_count, &bm, &bn);
   const int64_t mt = (a.M + bm - 1) / bm;
-  int bn = 256;
-  double best = -1.0;
-  const int cands[3] = {256, 192, 128};
-  const double eff[3] = {1.0, 0.9, 0.8};
-  for (int i = 0; i < 3; ++i) {
-    const double tiles = static_cast<double>(((a.N + cands[i] - 1) / cands[i]) * mt);
-    const double waves = tiles / d->sm_count;
-    const double score = eff[i] * waves / std::ceil(waves);
-    if (score > best + 1e-9) {
-      best = score;
-      bn = cands[i];
-    }
-  }
   CUtensorMap tm_x, tm_w;
   if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGemmBK,
                   static_cast<uint32_t>(bm), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
@@ -957,6 +968,73 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   return TB_ERR_SHAPE;
 }
 
+// ------------------------------------------------------------------ linear: integer-mode GEMM
+// Integer mode on the tensor cores from this many tokens (fewer: the plain
+// kernel, exact as well).
+constexpr int kGi8MinM = 16;
+
+bool gemm_i8_ok(const LinearArgs& a) {
+  if (a.xt != TB_INT8 || a.M < kGi8MinM || a.K % kGi8BK != 0 || (a.M + kGemmUM - 1) / kGemmUM > 65535 ||
+      a.N >= (int64_t(1) << 30))
+    return false;
+  if (!(aligned(a.x, 16) && aligned(a.packed, 16) && aligned(a.y, 16))) return false;
+  // base-3: re-encoded to 2-bit slots first, in a workspace the caller passed
+  if (a.f == TB_FMT_BASE3)
+    return a.ws != nullptr && aligned(a.ws, 16) && a.ws_bytes >= b3_transcode_bytes(a.f, a.M, a.N, a.K);
+  return true;
+}
+
+tb_status run_gemm_i8(const LinearArgs& a, const DevInfo* d) {
+  if (a.f == TB_FMT_BASE3) {
+    const int64_t ngroups = a.N * (a.K / 128);
+    transcode_b3_to_2bit_kernel<<<static_cast<unsigned>((ngroups + 255) / 256), 256, 0, a.st>>>(
+        a.packed, static_cast<uint4*>(a.ws), ngroups);
+    if (launch_status() != TB_OK) return TB_ERR_CUDA;
+    LinearArgs c = a;
+    c.f = TB_FMT_2BIT;
+    c.packed = static_cast<const uint8_t*>(a.ws);
+    return run_gemm_i8(c, d);
+  }
+  const bool one_bit = a.f == TB_FMT_1BIT;
+  int bm = 256, bn = 256;
+  gemm_tiles(a.M, a.N, d->sm_count, &bm, &bn);
+  CUtensorMap tm_x, tm_w;
+  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.x, a.K, a.M, a.K, kGi8BK, static_cast<uint32_t>(bm),
+                  CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+    return TB_ERR_CUDA;
+  const uint64_t wrow = one_bit ? a.K / 8 : a.K / 4;
+  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, wrow / 4, a.N, wrow,
+                  static_cast<uint32_t>(gi8_w_row_bytes(one_bit ? 2 : 0) / 4), static_cast<uint32_t>(bn)) != TB_OK)
+    return TB_ERR_CUDA;
+  GemmI8Params gp;
+  gp.M = static_cast<int>(a.M);
+  gp.N = static_cast<int>(a.N);
+  gp.K = static_cast<int>(a.K);
+  gp.y = static_cast<int32_t*>(a.y);
+  const dim3 grid(static_cast<unsigned>((a.N + bn - 1) / bn), static_cast<unsigned>((a.M + bm - 1) / bm));
+#define TB_GI8_F(BM, BN, F)                                                                                \
+  {                                                                                                        \
+    auto k = gemm_i8_kernel<BM, BN, F>;                                                                    \
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
+    return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gi8_smem_bytes(BM, BN, F)), a.st, tm_x, \
+                      tm_w, gp);                                                                           \
+  }
+#define TB_GI8(BM, BN)                \
+  if (bm == BM && bn == BN) {         \
+    if (one_bit) TB_GI8_F(BM, BN, 2)  \
+    TB_GI8_F(BM, BN, 0)               \
+  }
+  TB_GI8(256, 256)
+  TB_GI8(256, 192)
+  TB_GI8(256, 128)
+  TB_GI8(128, 256)
+  TB_GI8(128, 192)
+  TB_GI8(128, 128)
+#undef TB_GI8
+#undef TB_GI8_F
+  return TB_ERR_SHAPE;
+}
+
 bool known_format(int f) { return f == TB_FMT_2BIT || f == TB_FMT_BASE3 || f == TB_FMT_1BIT; }
 
 tb_status validate_linear(const LinearArgs& a) {
@@ -993,7 +1071,7 @@ tb_status linear_impl(const LinearArgs& a, int path) {
   if (st != TB_OK) return st;
   if (path == TB_PATH_AUTO) path = auto_path(a);
   if (path == TB_PATH_GEMV && !gemv_ok(a)) return TB_ERR_SHAPE;
-  if (path == TB_PATH_GEMM && !gemm_ok(a)) return TB_ERR_SHAPE;
+  if (path == TB_PATH_GEMM && !(a.xt == TB_INT8 ? gemm_i8_ok(a) : gemm_ok(a))) return TB_ERR_SHAPE;
   if (path == TB_PATH_GEMV_TC && !gemv_tc_ok(a)) return TB_ERR_SHAPE;
   if (path != TB_PATH_GEMV && path != TB_PATH_GEMM && path != TB_PATH_SIMPLE && path != TB_PATH_GEMV_TC)
     return TB_ERR_SHAPE;
@@ -1002,7 +1080,7 @@ tb_status linear_impl(const LinearArgs& a, int path) {
   if (st != TB_OK) return st;
   switch (path) {
     case TB_PATH_GEMV: return run_gemv(a, d);
-    case TB_PATH_GEMM: return run_gemm(a, d);
+    case TB_PATH_GEMM: return a.xt == TB_INT8 ? run_gemm_i8(a, d) : run_gemm(a, d);
     case TB_PATH_GEMV_TC: return run_gemv_tc(a, d);
     default: return run_simple(a);
   }

@@ -207,3 +207,14 @@ def test_path_selection_1bit(lib):
     assert p(tb.TB_BF16, "1bit", 1, 256, 640, has_signs=False) == tb.TB_PATH_SIMPLE
     assert p(tb.TB_INT8, "1bit", 4, 256, 1024, has_signs=False) == tb.TB_PATH_SIMPLE
     assert p(tb.TB_BF16, "1bit", 1, 17408, 5120, aligned16=False) == tb.TB_PATH_SIMPLE
+
+
+def test_path_selection_integer_mode(lib):
+    p = tb.tb_ternary_linear_path
+    # kind::i8 tensor-core GEMM from 16 tokens (any K % 128), else the plain kernel
+    assert p(tb.TB_INT8, "2bit", 16, 256, 1024, has_signs=False) == tb.TB_PATH_GEMM
+    assert p(tb.TB_INT8, "2bit", 15, 256, 1024, has_signs=False) == tb.TB_PATH_SIMPLE
+    assert p(tb.TB_INT8, "2bit", 2048, 17408, 5120, has_signs=False) == tb.TB_PATH_GEMM
+    assert p(tb.TB_INT8, "1bit", 2048, 17408, 640, has_signs=False) == tb.TB_PATH_GEMM
+    assert p(tb.TB_INT8, "base3", 64, 17408, 5120, has_signs=False) == tb.TB_PATH_GEMM
+    assert p(tb.TB_INT8, "2bit", 2048, 17408, 5120, has_signs=False, aligned16=False) == tb.TB_PATH_SIMPLE
