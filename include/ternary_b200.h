@@ -279,6 +279,17 @@ tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* p
  * fault recorded.  Synchronous (waits for the device's work to finish). */
 tb_status tb_get_device_fault(uint32_t* code, int clear);
 
+/* Failure-detection test hook (no counterpart on the pages).  With stall != 0
+ * the weight-copy producers of the one-token decode kernel and of the fp16
+ * GEMM issue nothing, so every wait for those copies runs out: the kernel
+ * records FAULT code 1 (a consumer gave up waiting for a stage) in the fault
+ * word, returns without hanging and leaves its output incomplete.
+ * wait_limit_ns sets how long a bounded wait lasts (0 = the default 2 s), for
+ * every kernel of the library on the current device.  Synchronous; call it
+ * between kernels, with nothing of the library in flight, and call it again
+ * with (0, 0) to restore normal operation. */
+tb_status tb_test_stall_copies(uint32_t stall, uint64_t wait_limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,6 +39,7 @@ _SIGNATURES = {
                                     _vp, _sz, _int, _vp]),
     "tb_ternary_linear_path": (_int, [_int, _int, _i64, _i64, _i64, _int, _int]),
     "tb_get_device_fault": (_int, [ctypes.POINTER(ctypes.c_uint32), _int]),
+    "tb_test_stall_copies": (_int, [ctypes.c_uint32, ctypes.c_uint64]),
     "tb_ternary_linear_noalloc": (_int, [_vp, _int, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _int,
                                          _vp]),
 }
@@ -186,3 +187,10 @@ def tb_get_device_fault(clear=False) -> int:
     v = ctypes.c_uint32(0)
     _done(load().tb_get_device_fault(ctypes.byref(v), int(clear)), "tb_get_device_fault", True)
     return v.value
+
+
+def tb_test_stall_copies(stall, wait_limit_ns=0):
+    """Failure-detection test hook (see the C header): with stall the weight
+    copies of the one-token decode and of the fp16 GEMM are not issued and the
+    waits for them run out after wait_limit_ns (0 = the default 2 s)."""
+    _done(load().tb_test_stall_copies(int(bool(stall)), int(wait_limit_ns)), "tb_test_stall_copies", True)

@@ -258,7 +258,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       prefetch_tensormap(&tm_x);
       prefetch_tensormap(&tm_w);
       pdl_wait();  // x' comes from the prep kernel
-      for (int kb = 0; kb < nk; ++kb) {
+      const bool stall = test_stall_copies();  // failure-detection test: no copies
+      for (int kb = 0; kb < nk && !stall; ++kb) {
         const int s = kb % kGemmStages;
         if (kb >= kGemmStages &&
             !mbar_wait(&empty[s], ((kb / kGemmStages) & 1) ^ 1, FAULT_WAIT_EMPTY))

@@ -499,12 +499,13 @@ __global__ void __launch_bounds__(kG1Threads, 2)
   const int pre = min(p.nslots, p.nstage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  const bool stall = test_stall_copies();  // failure-detection test: no weight copies
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tm_w);
     for (int s = 0; s < p.nstage; ++s) {
       mbar_init(&full[s], 1);
       done[s] = 0;
-      issued[s] = s < pre ? 1u : 0u;
+      issued[s] = s < pre && !stall ? 1u : 0u;
     }
     *cta_fault = 0;
     mbar_init(pre_bar, 1);
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(kG1Threads, 2)
         for (int b = 0; b < (p.K >> 10); ++b)
           bulk_load(act + b * 8 * kG1GroupStride, p.signs + static_cast<int64_t>(b) * kHB, kHB, pre_bar);
     }
-    for (int s = kG1Warps - 1 - warp; s < pre; s += kG1Warps)
+    for (int s = kG1Warps - 1 - warp; s < pre && !stall; s += kG1Warps)
       gemv1_issue<kFmt>(&tm_w, p, ring, &full[s], s, s, r0);
     if constexpr (!kFused) {
       if (warp == kG1Warps - 1) {

@@ -27,6 +27,20 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 // The library is one translation unit, so the fault word is defined here.
 __device__ uint32_t g_fault = 0;
 
+// Failure-detection test hook (tb_test_stall_copies): while bit 0 is set, the
+// TMA producers of the one-token decode and of the fp16 GEMM issue no weight
+// copies, so every wait for them runs out after g_wait_limit_ns.  Both words
+// are only ever written by the host between kernels.
+__device__ uint32_t g_test_stall = 0;
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+__device__ __forceinline__ bool test_stall_copies() {
+  return (*reinterpret_cast<volatile uint32_t*>(&g_test_stall) & 1u) != 0u;
+}
+__device__ __forceinline__ unsigned long long wait_limit_ns() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
+
 __device__ __forceinline__ void record_fault(uint32_t code) {
   atomicCAS(&g_fault, 0u, code);
 }
@@ -80,14 +94,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, records `fault` and returns false.
+// Waits for the phase with the given parity to complete.  Gives up after the
+// wait limit (2 s unless a test shortened it), records `fault` and returns
+// false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t fault) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
+  const unsigned long long limit = wait_limit_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit) {
       record_fault(fault);
       return false;
     }
@@ -100,10 +116,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, uint32_t fault) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
+  const unsigned long long limit = wait_limit_ns();
   for (;;) {
     __nanosleep(100);
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit) {
       record_fault(fault);
       return false;
     }

@@ -1324,6 +1324,17 @@ tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* p
   return run_gemv(a, d);
 }
 
+tb_status tb_test_stall_copies(uint32_t stall, uint64_t wait_limit_ns) {
+  const uint32_t v = stall ? 1u : 0u;
+  const unsigned long long lim = wait_limit_ns != 0 ? wait_limit_ns : tb::kWaitLimitNs;
+  if (cudaMemcpyToSymbol(tb::g_test_stall, &v, sizeof(v)) != cudaSuccess ||
+      cudaMemcpyToSymbol(tb::g_wait_limit_ns, &lim, sizeof(lim)) != cudaSuccess) {
+    cudaGetLastError();
+    return TB_ERR_CUDA;
+  }
+  return TB_OK;
+}
+
 tb_status tb_get_device_fault(uint32_t* code, int clear) {
   if (code == nullptr) return TB_ERR_NULL;
   if (cudaMemcpyFromSymbol(code, tb::g_fault, sizeof(uint32_t)) != cudaSuccess) {
