@@ -121,10 +121,13 @@ typedef int tb_path;
 #define TB_PATH_SIMPLE 3 /* plain per-row kernel: any K % 128, any alignment    */
 #define TB_PATH_GEMV_TC 4 /* tcgen05 decode kernel (codes unpacked into TMEM as
                             the u8 A operand, int8 activation planes as B in
-                            shared memory), for M <= 16 and N <= 148 * 128;
-                            base-3 with 8-16 tokens is first re-encoded to 2-bit
-                            slots in the workspace.  Chosen by TB_PATH_AUTO from
-                            4 tokens (2-bit) or 8 tokens (base-3)               */
+                            shared memory, per-group int32 sums read back and
+                            scaled), for M <= 16, any N; K is split over CTAs
+                            when rows are few (partial sums in the workspace,
+                            added in a fixed order).  base-3 with 8-16 tokens is
+                            first re-encoded to 2-bit slots in the workspace.
+                            Chosen by TB_PATH_AUTO from 4 tokens (2-bit) or 8
+                            tokens (base-3)                                    */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* tb_status_string(tb_status st);

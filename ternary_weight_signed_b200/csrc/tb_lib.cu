@@ -223,6 +223,14 @@ size_t workspace_bytes(int64_t M, int64_t K) {
   return (b + 255) & ~static_cast<size_t>(255);
 }
 
+size_t gtc_extra_bytes(int f, int64_t M, int64_t N, int64_t K);
+
+// Everything a call may use: the activations of any path, the base-3
+// re-encoding, the tensor-core decode's partial sums and counters.
+size_t required_ws(int f, int64_t M, int64_t N, int64_t K) {
+  return workspace_bytes(M, K) + b3_transcode_bytes(f, M, N, K) + gtc_extra_bytes(f, M, N, K);
+}
+
 bool fast_aligned(const LinearArgs& a) {
   return aligned(a.packed, 16) && aligned(a.scales, 16) && aligned(a.x, 16) && aligned(a.y, 16) &&
          aligned(a.ws, 16) && (a.signs == nullptr || aligned(a.signs, 16));
@@ -405,50 +413,64 @@ bool b3_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, B3Plan
 }
 
 struct GtcPlan {
-  int grid, box_rows, rows_box, parts, gpp, nb, nstages, depth;
-  uint32_t w_box_bytes, box_stride, part_bytes, stage_bytes, tmem_cols;
-  size_t smem;
+  int grid, R, T, S, nblk, gbox, nstages, ntiles;
+  uint32_t box_stride, stage_bytes;
+  GtcLayout lay;
 };
 
 // Geometry of the tensor-core decode kernel; false if these sizes do not fit it.
+// Tiles of up to 128 rows (one per TMEM lane, at least 16).  With no more
+// than sm_count tiles of 128 rows, K is split over S CTAs per tile so that
+// tiles x S fills the SMs (each tile's activations are still read once); with
+// more, a CTA runs T tiles in turn.
 bool gtc_plan(int64_t M, int64_t N, int64_t K, int sm_count, int max_smem, GtcPlan* out) {
-  if (M < 1 || M > kGtcMaxM || K % 1024 != 0 || N < 1) return false;
+  if (M < 1 || M > kGtcMaxM || K % 1024 != 0 || K < 1024 || N < 1 || sm_count < 1) return false;
   GtcPlan pl;
-  pl.grid = static_cast<int>(N < sm_count ? N : sm_count);
-  pl.box_rows = static_cast<int>((N + pl.grid - 1) / pl.grid);
-  if (pl.box_rows > 128) return false;
-  pl.rows_box = 32 * ((pl.box_rows + 31) / 32);
-  const int G = static_cast<int>(K / 128);
-  const int AR = gtc_atom_rows(static_cast<int>(M));  // D columns per step
-  int parts = 128 / pl.rows_box;
-  if (parts > 3) parts = 3;  // TMEM: depth x (32 parts + AR) columns with depth >= 4
-  if (parts > G / 4) parts = G / 4;
-  if (parts < 1) parts = 1;
-  pl.gpp = 4 * ((G + 4 * parts - 1) / (4 * parts));
-  pl.parts = (G + pl.gpp - 1) / pl.gpp;
-  pl.depth = 8;  // a multiple of the 4 step groups
-  if (pl.depth * (32 * pl.parts + AR) > 512) pl.depth = 4;
-  const int cols = pl.depth * (32 * pl.parts + AR);
-  if (cols > 512) return false;
-  pl.tmem_cols = 32;
-  while (static_cast<int>(pl.tmem_cols) < cols) pl.tmem_cols <<= 1;
-  pl.w_box_bytes = static_cast<uint32_t>(pl.box_rows) * 128u;
-  pl.box_stride = (pl.w_box_bytes + 1023u) & ~1023u;
-  for (pl.nb = 2; pl.nb >= 1; --pl.nb) {
-    pl.part_bytes = pl.nb * pl.box_stride + 4u * pl.nb * static_cast<uint32_t>(gtc_atom_bytes(static_cast<int>(M)));
-    pl.stage_bytes = static_cast<uint32_t>(pl.parts) * pl.part_bytes;
-    const int64_t fixed = gtc_smem_bytes(static_cast<int>(M), K, pl.box_rows, 0, 0, pl.depth) + 8 * 2 * 6;
-    int64_t ns = (static_cast<int64_t>(max_smem) - fixed) / pl.stage_bytes;
-    if (ns > 6) ns = 6;
-    if (ns >= 2) {
-      pl.nstages = static_cast<int>(ns);
-      pl.smem = static_cast<size_t>(
-          gtc_smem_bytes(static_cast<int>(M), K, pl.box_rows, pl.stage_bytes, pl.nstages, pl.depth));
-      *out = pl;
-      return true;
-    }
+  pl.nblk = static_cast<int>(K / 1024);
+  const int64_t tiles128 = (N + kGtcMaxRows - 1) / kGtcMaxRows;
+  int64_t tiles;
+  if (tiles128 <= sm_count) {
+    pl.T = 1;
+    pl.S = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>(std::min<int64_t>(pl.nblk, kGtcMaxSplits), sm_count / tiles128)));
+    tiles = std::min<int64_t>(sm_count / pl.S, (N + 15) / 16);
+    pl.R = static_cast<int>((N + tiles - 1) / tiles);
+  } else {
+    pl.S = 1;
+    const int64_t per_cta = (N + sm_count - 1) / sm_count;
+    pl.T = static_cast<int>((per_cta + kGtcMaxRows - 1) / kGtcMaxRows);
+    pl.R = static_cast<int>((per_cta + pl.T - 1) / pl.T);
   }
-  return false;
+  tiles = (N + pl.R - 1) / pl.R;
+  pl.ntiles = static_cast<int>(tiles);
+  const int64_t groups = (tiles + pl.T - 1) / pl.T;
+  if (groups * pl.S > 2147483647LL) return false;
+  pl.grid = static_cast<int>(groups * pl.S);
+  pl.gbox = 8 * ((pl.nblk + pl.S - 1) / pl.S);
+  if (pl.gbox > 256 || pl.R > kGtcMaxRows) return false;  // TMA box limits
+  pl.box_stride = static_cast<uint32_t>(align_up(static_cast<int64_t>(pl.R) * 128, 1024));
+  pl.stage_bytes = pl.box_stride + 4u * static_cast<uint32_t>(gtc_atom_bytes(static_cast<int>(M)));
+  const int MT = gtc_capacity(static_cast<int>(M));  // info and sums sized for the kernel's token capacity
+  const GtcLayout l0 = gtc_layout(MT, pl.R, pl.T, pl.gbox, 0, pl.stage_bytes);
+  int64_t ns = (max_smem - l0.bytes - 64) / pl.stage_bytes;
+  if (ns > 8) ns = 8;
+  if (ns < 2) return false;
+  pl.nstages = static_cast<int>(ns);
+  pl.lay = gtc_layout(MT, pl.R, pl.T, pl.gbox, pl.nstages, pl.stage_bytes);
+  if (pl.lay.bytes > max_smem) return false;
+  *out = pl;
+  return true;
+}
+
+// Workspace of the tensor-core decode beyond its activations: the K splits'
+// partial sums [S][M][N] fp32 and one counter per tile.  A bound over every
+// plan (S <= min(K / 1024, kGtcMaxSplits); tiles of 16 rows or more).
+size_t gtc_extra_bytes(int f, int64_t M, int64_t N, int64_t K) {
+  if (M > kGtcMaxM || K % 1024 != 0 || (f != TB_FMT_2BIT && f != TB_FMT_BASE3)) return 0;
+  const int64_t smax = std::min<int64_t>(K / 1024, kGtcMaxSplits);
+  const size_t part = static_cast<size_t>(smax * M * N * 4);
+  const size_t cnt = static_cast<size_t>(4 * ((N + 15) / 16));
+  return ((part + 255) & ~static_cast<size_t>(255)) + ((cnt + 255) & ~static_cast<size_t>(255));
 }
 
 constexpr int kB200Sms = 148;
@@ -654,45 +676,58 @@ tb_status run_gemv_typed(const LinearArgs& a, const DevInfo* d) {
 template <typename TIn>
 tb_status run_gemv_tc_typed(const LinearArgs& a, const DevInfo* d, const GtcPlan& pl) {
   uint8_t* act = static_cast<uint8_t*>(a.ws);
+  const size_t act_bytes = (static_cast<size_t>(gtc_ws_bytes(a.M, a.K)) + 255) & ~static_cast<size_t>(255);
+  float* part = reinterpret_cast<float*>(act + act_bytes);
+  const size_t part_bytes =
+      (static_cast<size_t>(pl.S) * a.M * a.N * 4 + 255) & ~static_cast<size_t>(255);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(act + act_bytes + part_bytes);
+  if (act_bytes + part_bytes + 4 * static_cast<size_t>(pl.ntiles) > a.ws_bytes) return TB_ERR_WORKSPACE;
   const dim3 pgrid(static_cast<unsigned>(a.M), static_cast<unsigned>(a.K / kHB));
+  // a plain launch: measured on B200, letting it start early under the
+  // previous decode kernel cost 2-4 us per call
   prep_gemv_tc_kernel<TIn><<<pgrid, kHThreads, 0, a.st>>>(static_cast<const TIn*>(a.x), a.signs, act, a.K,
-                                                          static_cast<int>(a.M));
+                                                          static_cast<int>(a.M), cnt, pl.S > 1 ? pl.ntiles : 0);
   if (launch_status() != TB_OK) return TB_ERR_CUDA;
-  CUtensorMap tm_w;
+  CUtensorMap tm_w, tm_s;
   if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.K / 16, a.N, a.K / 4, 32,
-                  static_cast<uint32_t>(pl.box_rows), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+                  static_cast<uint32_t>(pl.R), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+    return TB_ERR_CUDA;
+  if (make_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.scales, a.K / 128, a.N, (a.K / 128) * 2,
+                  static_cast<uint32_t>(pl.gbox), static_cast<uint32_t>(pl.R)) != TB_OK)
     return TB_ERR_CUDA;
   GemvTcParams p;
   p.act = act;
-  p.scales = a.scales;
   p.y = a.y;
+  p.part = part;
+  p.cnt = cnt;
   p.M = static_cast<int>(a.M);
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
-  p.box_rows = pl.box_rows;
-  p.rows_box = pl.rows_box;
-  p.parts = pl.parts;
-  p.gpp = pl.gpp;
-  p.nb = pl.nb;
+  p.G = static_cast<int>(a.K / 128);
+  p.R = pl.R;
+  p.T = pl.T;
+  p.S = pl.S;
+  p.nblk = pl.nblk;
+  p.gbox = pl.gbox;
+  p.sc_tile = static_cast<int>(gtc_sc_tile_bytes(pl.R, pl.gbox) / 2);
   p.nstages = pl.nstages;
-  p.depth = pl.depth;
-  p.depth_log2 = pl.depth == 8 ? 3 : 2;
-  p.gps_log2 = pl.nb == 2 ? 3 : 2;
-  p.w_box_bytes = pl.w_box_bytes;
   p.box_stride = pl.box_stride;
-  p.part_bytes = pl.part_bytes;
   p.stage_bytes = pl.stage_bytes;
-  p.tmem_cols = pl.tmem_cols;
-#define TB_GTC_CASE(MM)                                                                \
-  case MM:                                                                             \
-    if (a.yt == TB_FP32) {                                                             \
-      auto k = gemv_tc_kernel<MM, float>;                                              \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                               \
-      return launch_pdl(k, dim3(pl.grid), dim3(kGtcThreads), pl.smem, a.st, tm_w, p);  \
-    } else {                                                                           \
-      auto k = gemv_tc_kernel<MM, __nv_bfloat16>;                                      \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                               \
-      return launch_pdl(k, dim3(pl.grid), dim3(kGtcThreads), pl.smem, a.st, tm_w, p);  \
+  p.off_sc = pl.lay.off_sc;
+  p.off_info = pl.lay.off_info;
+  p.off_red = pl.lay.off_red;
+  p.off_bar = pl.lay.off_bar;
+  const size_t smem = static_cast<size_t>(pl.lay.bytes);
+#define TB_GTC_CASE(MM)                                                                          \
+  case MM:                                                                                       \
+    if (a.yt == TB_FP32) {                                                                       \
+      auto k = gemv_tc_kernel<MM, float>;                                                        \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                         \
+      return launch_pdl(k, dim3(pl.grid), dim3(kGtcThreads), smem, a.st, tm_w, tm_s, p);         \
+    } else {                                                                                     \
+      auto k = gemv_tc_kernel<MM, __nv_bfloat16>;                                                \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                         \
+      return launch_pdl(k, dim3(pl.grid), dim3(kGtcThreads), smem, a.st, tm_w, tm_s, p);         \
     }
   switch (gtc_capacity(static_cast<int>(a.M))) {
     TB_GTC_CASE(4)
@@ -1059,8 +1094,7 @@ tb_status validate_linear(const LinearArgs& a) {
   if (a.signs != nullptr && !aligned(a.signs, 8)) return TB_ERR_ALIGN;
   if (a.f == TB_FMT_BASE3 && !aligned(a.packed, 2)) return TB_ERR_ALIGN;
   if (!int_mode) {
-    if (a.ws == nullptr || a.ws_bytes < workspace_bytes(a.M, a.K) + b3_transcode_bytes(a.f, a.M, a.N, a.K))
-      return TB_ERR_WORKSPACE;
+    if (a.ws == nullptr || a.ws_bytes < required_ws(a.f, a.M, a.N, a.K)) return TB_ERR_WORKSPACE;
     if (!aligned(a.ws, 16)) return TB_ERR_ALIGN;
   }
   return TB_OK;
@@ -1226,7 +1260,7 @@ tb_status tb_prepare_weights(const void* w, tb_dtype wt, const int8_t* signs, in
 
 size_t tb_ternary_linear_workspace(tb_format f, int64_t M, int64_t N, int64_t K) {
   if (!known_format(f) || M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
-  return workspace_bytes(M, K) + b3_transcode_bytes(f, M, N, K);
+  return required_ws(f, M, N, K);
 }
 
 tb_status tb_ternary_linear_ex(const void* x, tb_dtype xt, const uint8_t* packed, const uint16_t* scales,
@@ -1253,7 +1287,7 @@ int tb_ternary_linear_path(tb_dtype xt, tb_format f, int64_t M, int64_t N, int64
                has_signs ? reinterpret_cast<const int8_t*>(0x2000) : nullptr,
                reinterpret_cast<void*>(0x3000), xt == TB_INT8 ? TB_INT32 : TB_FP32,
                reinterpret_cast<void*>(0x4000),
-               workspace_bytes(M > 0 ? M : 1, K > 0 ? K : 128) + b3_transcode_bytes(f, M, N, K), nullptr};
+               required_ws(f, M > 0 ? M : 1, N > 0 ? N : 1, K > 0 ? K : 128), nullptr};
   if (validate_linear(a) != TB_OK) return -1;
   return auto_path(a);
 }
@@ -1302,8 +1336,8 @@ tb_status tb_ternary_linear_noalloc(const void* x, tb_dtype xt, const uint8_t* p
   // Validate as tb_ternary_linear would with an ample aligned workspace, then
   // check the fixed scratch's limit and the GEMV path's own rules.
   LinearArgs a{x, xt, packed, scales, TB_FMT_2BIT, M, N, K, signs, y, yt,
-               reinterpret_cast<void*>(static_cast<uintptr_t>(256)), workspace_bytes(M > 0 ? M : 1, K > 0 ? K : 128),
-               as_stream(stream)};
+               reinterpret_cast<void*>(static_cast<uintptr_t>(256)),
+               required_ws(TB_FMT_2BIT, M > 0 ? M : 1, N > 0 ? N : 1, K > 0 ? K : 128), as_stream(stream)};
   tb_status st = validate_linear(a);
   if (st != TB_OK) return st;
   if (xt == TB_INT8) return TB_ERR_DTYPE;

@@ -1,7 +1,7 @@
 """Runs one named workload through tb_ternary_linear a few times, for profilers.
 
     python -m ternary_weight_signed_b200.profile_case --workload gemv_gateup_k5120_n17408 \
-        [--m 1] [--fmt 2bit|base3] [--path auto|gemv|gemm|simple] [--reps 4]
+        [--m 1] [--fmt 2bit|base3|1bit] [--path auto|gemv|gemv_tc|gemm|simple] [--reps 4]
 
 Inputs are the seeded synthetic ones of the workload; nothing is checked here
 (the tests do that).  Exits non-zero if a call fails or the device records a
@@ -25,8 +25,8 @@ def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="gemv_gateup_k5120_n17408", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--m", type=int, default=None)
-    ap.add_argument("--fmt", default="2bit", choices=["2bit", "base3"])
-    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm", "simple"])
+    ap.add_argument("--fmt", default="2bit", choices=["2bit", "base3", "1bit"])
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemv_tc", "gemm", "simple"])
     ap.add_argument("--yt", default="fp32", choices=["fp32", "bf16"])
     ap.add_argument("--reps", type=int, default=4)
     a = ap.parse_args(argv)
@@ -34,7 +34,8 @@ def main(argv=None) -> int:
     w = inputs.WORKLOADS[a.workload]
     m = a.m or w["ms"][0]
     n, k = w["n"], w["k"]
-    p = inputs.make_linear_inputs(w["seed"], m, n, k, w["p0"], w["scale_kind"], w["outlier_rate"])
+    p0 = 0.0 if a.fmt == "1bit" else w["p0"]  # 1-bit codes are -1 or +1
+    p = inputs.make_linear_inputs(w["seed"], m, n, k, p0, w["scale_kind"], w["outlier_rate"])
     dev = torch.device("cuda:0")
     codes = torch.from_numpy(p.codes).to(dev)
     packed = torch.empty(tb.tb_packed_bytes(a.fmt, n, k), dtype=torch.uint8, device=dev)
@@ -46,7 +47,7 @@ def main(argv=None) -> int:
     y = torch.empty(m, n, dtype=torch.float32 if a.yt == "fp32" else torch.bfloat16, device=dev)
     ws_bytes = tb.tb_ternary_linear_workspace(a.fmt, m, n, k)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    path = {"auto": tb.TB_PATH_AUTO, "gemv": tb.TB_PATH_GEMV, "gemm": tb.TB_PATH_GEMM,
+    path = {"auto": tb.TB_PATH_AUTO, "gemv": tb.TB_PATH_GEMV, "gemv_tc": tb.TB_PATH_GEMV_TC, "gemm": tb.TB_PATH_GEMM,
             "simple": tb.TB_PATH_SIMPLE}[a.path]
     for _ in range(a.reps):
         tb.tb_ternary_linear_ex(x, tb.TB_BF16, packed, scales, a.fmt, m, n, k, signs, y, yt, ws,

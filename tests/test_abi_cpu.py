@@ -131,11 +131,11 @@ def test_path_selection(lib):
     assert p(tb.TB_BF16, "base3", 16, 5120, 17408) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "base3", 17, 5120, 17408) == tb.TB_PATH_GEMM
     assert p(tb.TB_BF16, "base3", 2048, 17408, 5120) == tb.TB_PATH_GEMM
-    # more weight rows than the tensor-core decode takes (148 x 128): 8-16 base-3
-    # tokens go to the re-encoded GEMM, 4 two-bit tokens to the CUDA-core decode
-    assert p(tb.TB_BF16, "base3", 16, 34816, 5120) == tb.TB_PATH_GEMM
-    assert p(tb.TB_BF16, "base3", 8, 19000, 1024) == tb.TB_PATH_GEMM
-    assert p(tb.TB_BF16, "2bit", 4, 34816, 5120) == tb.TB_PATH_GEMV
+    # more weight rows than 148 x 128: the tensor-core decode runs two row
+    # tiles per CTA
+    assert p(tb.TB_BF16, "base3", 16, 34816, 5120) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "base3", 8, 19000, 1024) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "2bit", 4, 34816, 5120) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "2bit", 1, 256, 1000) == -1
 
 

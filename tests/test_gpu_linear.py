@@ -245,12 +245,14 @@ def test_gemm_base3_via_reencoding(m):
     _check(prob.linear(AUTO), ref, prob.p)
 
 
-def test_base3_tokens_beyond_tensor_core_rows_take_the_gemm():
-    """12 base-3 tokens and more rows than the tensor-core decode takes: the
-    automatic path re-encodes to 2-bit slots and runs the GEMM."""
-    assert tb.tb_ternary_linear_path(tb.TB_BF16, "base3", 12, 19000, 1024, True, True) == GEMM
+def test_base3_tokens_beyond_one_row_tile_per_sm():
+    """12 base-3 tokens and more rows than 148 x 128: re-encoded to 2-bit slots,
+    then the tensor-core decode with two row tiles per CTA (automatic path) or
+    the GEMM (asked for)."""
+    assert tb.tb_ternary_linear_path(tb.TB_BF16, "base3", 12, 19000, 1024, True, True) == tb.TB_PATH_GEMV_TC
     prob, ref = _problem(28, 12, 19000, 1024, 0.33, "base3", "abs_normal", 0.01)
     _check(prob.linear(AUTO), ref, prob.p)
+    _check(prob.linear(GEMM), ref, prob.p)
 
 
 @pytest.mark.parametrize("yt", [tb.TB_FP32, tb.TB_BF16])
@@ -301,8 +303,9 @@ def test_gemm_invalid_bytes_no_fault():
 GEMV_TC = tb.TB_PATH_GEMV_TC
 
 
-# shapes within the tensor-core decode kernel's limit of 148 x 128 rows
-GEMV_TC_CASES = [c for c in WORKLOAD_CASES if c[2] <= 148 * 128]
+# every workload shape: the tensor-core decode takes any N (two or more row
+# tiles per CTA beyond 148 x 128 rows) and splits K over CTAs when rows are few
+GEMV_TC_CASES = WORKLOAD_CASES
 
 
 @pytest.mark.parametrize("case", GEMV_TC_CASES, ids=lambda c: f"m{c[1]}n{c[2]}k{c[3]}")
@@ -334,14 +337,30 @@ def test_base3_reencoded_tensor_core_decode(m):
     _check(prob.linear(AUTO), ref, prob.p)
 
 
-def test_gemv_tensor_core_rejects_rows_beyond_tmem():
-    """More rows than 148 CTAs x 128 TMEM lanes: the tensor-core decode kernel
-    refuses the shape; the CUDA-core kernel takes it."""
-    prob, ref = _problem(24, 2, 20480, 1024, 0.33, "2bit")
-    ws_bytes = tb.tb_ternary_linear_workspace("2bit", 2, 20480, 1024)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=DEV)
-    st = tb.tb_ternary_linear_ex(prob.x, tb.TB_BF16, prob.packed, prob.scales, "2bit", 2, 20480,
-                                 1024, prob.signs, torch.empty(2, 20480, device=DEV), tb.TB_FP32,
-                                 ws, ws_bytes, GEMV_TC, check=False)
-    assert st == tb.TB_ERR_SHAPE
-    _check(prob.linear(GEMV), ref, prob.p)
+@pytest.mark.parametrize("m", [2, 16])
+@pytest.mark.parametrize("n", [20480, 34816])
+def test_gemv_tensor_core_rows_beyond_one_tile_per_sm(n, m):
+    """More rows than 148 CTAs x 128 TMEM lanes: each CTA runs two row tiles in
+    turn (34816 = the gate|up pair stacked along N)."""
+    prob, ref = _problem(24, m, n, 1024 if n == 20480 else 5120, 0.33, "2bit")
+    _check(prob.linear(GEMV_TC), ref, prob.p)
+
+
+@pytest.mark.parametrize("m", [1, 3, 4, 8, 16])
+@pytest.mark.parametrize("n,k", [(5120, 17408), (1024, 5120), (256, 1024), (6144, 5120), (5120, 6144)])
+def test_gemv_tensor_core_k_split(n, k, m):
+    """Few rows: K is split over several CTAs per row tile and the last CTA of
+    a tile adds the partial sums (down, k/v, tiny, q and o shapes)."""
+    prob, ref = _problem(27, m, n, k, 0.5, "2bit", "lognormal", 0.0)
+    _check(prob.linear(GEMV_TC), ref, prob.p)
+
+
+@pytest.mark.parametrize("n,k,m", [(5120, 17408, 16), (17408, 5120, 4), (34816, 5120, 8)])
+def test_gemv_tensor_core_repeatable(n, k, m):
+    """The split-K reduction adds the partial sums in a fixed order: repeated
+    calls agree bit for bit."""
+    prob, ref = _problem(28, m, n, k, 0.33, "2bit")
+    a = prob.linear(GEMV_TC)
+    b = prob.linear(GEMV_TC)
+    assert np.array_equal(a, b)
+    _check(a, ref, prob.p)
