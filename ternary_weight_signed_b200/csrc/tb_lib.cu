@@ -528,10 +528,13 @@ int auto_path(const LinearArgs& a) {
     if (gemv_ok(a)) return TB_PATH_GEMV;
     return gemm_ok(a) ? TB_PATH_GEMM : TB_PATH_SIMPLE;
   }
-  // 2-bit: the dp4a kernel's cost grows with M, the tensor-core one's hardly
-  // does; measured on B200 (K=17408, N=5120) the tensor-core kernel wins from
-  // 4 tokens on (31 us against 40 us).
-  if (a.f == TB_FMT_2BIT && a.M >= 4 && gemv_tc_ok(a)) return TB_PATH_GEMV_TC;
+  // 2-bit: the one-token kernel where it is preferred (it rotates x itself
+  // and overlaps consecutive calls), else the tensor-core decode, whose cost
+  // hardly grows with M.  Measured on B200: 2 tokens 13.9 against 17.6 us
+  // (17408 x 5120) and 17.8 against 24.9 us (5120 x 17408); one token on the
+  // long-K down shape 16.5 against 18.7 us.
+  if (a.f == TB_FMT_2BIT && !(a.M == 1 && g1_preferred(a.N, a.K, kB200Sms)) && gemv_tc_ok(a))
+    return TB_PATH_GEMV_TC;
   if (gemv_ok(a)) return TB_PATH_GEMV;       // M <= 4 (2-bit), M <= 7 (base-3)
   if (gemv_tc_ok(a)) return TB_PATH_GEMV_TC;  // up to 16 tokens (base-3 re-encoded)
   if (gemm_ok(a)) return TB_PATH_GEMM;

@@ -115,7 +115,11 @@ def test_linear_validation(lib):
 def test_path_selection(lib):
     p = tb.tb_ternary_linear_path
     assert p(tb.TB_BF16, "2bit", 1, 17408, 5120) == tb.TB_PATH_GEMV
-    assert p(tb.TB_BF16, "2bit", 3, 5120, 17408) == tb.TB_PATH_GEMV
+    # one token with long K and few rows (down shape), and 2-16 tokens: the
+    # tensor-core decode
+    assert p(tb.TB_BF16, "2bit", 1, 5120, 17408) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "2bit", 2, 17408, 5120) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "2bit", 3, 5120, 17408) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "2bit", 4, 5120, 17408) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "2bit", 1, 256, 1152, has_signs=False) == tb.TB_PATH_SIMPLE
     assert p(tb.TB_BF16, "2bit", 1, 17408, 5120, aligned16=False) == tb.TB_PATH_SIMPLE
@@ -136,6 +140,7 @@ def test_path_selection(lib):
     assert p(tb.TB_BF16, "base3", 16, 34816, 5120) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "base3", 8, 19000, 1024) == tb.TB_PATH_GEMV_TC
     assert p(tb.TB_BF16, "2bit", 4, 34816, 5120) == tb.TB_PATH_GEMV_TC
+    assert p(tb.TB_BF16, "2bit", 1, 34816, 5120) == tb.TB_PATH_GEMV
     assert p(tb.TB_BF16, "2bit", 1, 256, 1000) == -1
 
 

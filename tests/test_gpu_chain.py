@@ -19,16 +19,21 @@ pytestmark = pytest.mark.gpu
 
 STEPS = 6
 
-# format, tokens M, K (= N, so that y can be the next x), x/y dtype, path taken
+# format, tokens M, K (= N, so that y can be the next x), x/y dtype, path
+# asked for, and whether it is also the automatic choice
 CASES = [
-    ("2bit", 1, 5120, "bf16", tb.TB_PATH_GEMV),    # one launch, rotation inside
-    ("2bit", 1, 5120, "fp32", tb.TB_PATH_GEMV),
-    ("2bit", 1, 10240, "bf16", tb.TB_PATH_GEMV),   # activation kernel, then decode
-    ("2bit", 2, 5120, "bf16", tb.TB_PATH_GEMV),
-    ("2bit", 4, 5120, "bf16", tb.TB_PATH_GEMV_TC),
-    ("2bit", 64, 5120, "bf16", tb.TB_PATH_GEMM),
-    ("base3", 1, 5120, "bf16", tb.TB_PATH_GEMV),
-    ("base3", 8, 5120, "bf16", tb.TB_PATH_GEMV_TC),
+    ("2bit", 1, 5120, "bf16", tb.TB_PATH_GEMV, True),     # one launch, rotation inside
+    ("2bit", 1, 5120, "fp32", tb.TB_PATH_GEMV, True),
+    ("2bit", 1, 10240, "bf16", tb.TB_PATH_GEMV, True),    # activation kernel, then decode
+    ("2bit", 2, 5120, "bf16", tb.TB_PATH_GEMV, False),    # CUDA-core decode for two tokens
+    ("2bit", 2, 5120, "bf16", tb.TB_PATH_GEMV_TC, True),
+    ("2bit", 4, 5120, "bf16", tb.TB_PATH_GEMV_TC, True),
+    ("2bit", 16, 5120, "bf16", tb.TB_PATH_GEMV_TC, True),
+    ("2bit", 64, 5120, "bf16", tb.TB_PATH_GEMM, True),
+    ("base3", 1, 5120, "bf16", tb.TB_PATH_GEMV, True),
+    ("base3", 8, 5120, "bf16", tb.TB_PATH_GEMV_TC, True),
+    ("1bit", 1, 5120, "bf16", tb.TB_PATH_GEMV, True),
+    ("1bit", 4, 5120, "bf16", tb.TB_PATH_GEMM, True),
 ]
 
 DT = {"bf16": (tb.TB_BF16, torch.bfloat16), "fp32": (tb.TB_FP32, torch.float32)}
@@ -42,7 +47,7 @@ def _lib():
     assert tb.tb_get_device_fault() == 0
 
 
-def _chain(x0, layers, fmt, m, k, code, nbuf, sync):
+def _chain(x0, layers, fmt, m, k, code, nbuf, sync, path):
     """STEPS calls, call i on layer i % 2 from buffer i % nbuf into buffer
     (i + 1) % nbuf: nbuf = 2 is a ping-pong (each call also overwrites what the
     call before it read), nbuf = STEPS + 1 keeps every output.  Nothing but the
@@ -55,29 +60,29 @@ def _chain(x0, layers, fmt, m, k, code, nbuf, sync):
     for i in range(STEPS):
         packed, scales, signs = layers[i % 2]
         x, y = bufs[i % nbuf], bufs[(i + 1) % nbuf]
-        tb.tb_ternary_linear(x, code, packed, scales, fmt, m, k, k, signs, y, code, ws, ws_bytes,
-                             stream=stream.cuda_stream)
+        tb.tb_ternary_linear_ex(x, code, packed, scales, fmt, m, k, k, signs, y, code, ws, ws_bytes, path,
+                                stream=stream.cuda_stream)
         if sync:
             stream.synchronize()
     stream.synchronize()
     return [b.float().cpu().numpy() for b in bufs]
 
 
-@pytest.mark.parametrize("fmt,m,k,dtype,path", CASES)
-def test_chain_matches_synchronised_chain(fmt, m, k, dtype, path):
+@pytest.mark.parametrize("fmt,m,k,dtype,path,auto", CASES)
+def test_chain_matches_synchronised_chain(fmt, m, k, dtype, path, auto):
     code, tdt = DT[dtype]
-    assert tb.tb_ternary_linear_path(code, fmt, m, k, k) == path
+    assert (tb.tb_ternary_linear_path(code, fmt, m, k, k) == path) == auto
     layers = []
     for seed in (71, 72):
-        p = inputs.make_linear_inputs(seed, m, k, k, 0.33, "abs_normal", 0.01)
+        p = inputs.make_linear_inputs(seed, m, k, k, 0.0 if fmt == "1bit" else 0.33, "abs_normal", 0.01)
         packed, cnt = pack_dev(fmt, to_dev_codes(p.codes), k, k)
         assert int(cnt.item()) == 0
         layers.append((packed, to_dev_scales(p.scales), to_dev_codes(p.signs)))
         if seed == 71:
             x0 = torch.from_numpy(p.x).to(DEV).to(tdt)  # x drawn in float64, rounded like the bf16 inputs
     for nbuf in (STEPS + 1, 2):
-        free = _chain(x0, layers, fmt, m, k, code, nbuf, sync=False)
-        ref = _chain(x0, layers, fmt, m, k, code, nbuf, sync=True)
+        free = _chain(x0, layers, fmt, m, k, code, nbuf, False, path)
+        ref = _chain(x0, layers, fmt, m, k, code, nbuf, True, path)
         for i, (a, b) in enumerate(zip(free, ref)):
             assert np.all(np.isfinite(b)) and np.any(b != 0), f"buffer {i}: degenerate output"
             np.testing.assert_array_equal(a, b, err_msg=f"{nbuf} buffers: buffer {i} differs from the "
