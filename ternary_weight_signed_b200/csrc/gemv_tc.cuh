@@ -586,15 +586,24 @@ __global__ void __launch_bounds__(kGtcThreads, 1)
           }
           asm volatile("bar.sync 1, 256;" ::: "memory");
           if (*last_flag != 0u && live && team == 0) {
-            // the last CTA of the tile: add the S partial sums in split order
+            // The last CTA of the tile adds the S partial sums in split order.
+            // Every split's MT loads are independent and issued together (a
+            // dependent load per split and token measured 10 us per tile).
+            float v[MT];
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              if (m < M) {
-                float v = 0.f;
-                for (int s2 = 0; s2 < p.S; ++s2) v += __ldcg(&p.part[(static_cast<int64_t>(s2) * M + m) * p.N + n]);
-                y[static_cast<int64_t>(m) * p.N + n] = from_f32<TOut>(v);
-              }
+            for (int m = 0; m < MT; ++m) v[m] = 0.f;
+#pragma unroll 4
+            for (int s2 = 0; s2 < p.S; ++s2) {
+              const float* src = p.part + static_cast<int64_t>(s2) * M * p.N + n;
+              float pv[MT];
+#pragma unroll
+              for (int m = 0; m < MT; ++m) pv[m] = m < M ? __ldcg(src + static_cast<int64_t>(m) * p.N) : 0.f;
+#pragma unroll
+              for (int m = 0; m < MT; ++m) v[m] += pv[m];
             }
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+              if (m < M) y[static_cast<int64_t>(m) * p.N + n] = from_f32<TOut>(v[m]);
           }
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");  // the exchange buffer is free again
