@@ -1,0 +1,399 @@
+// Prefill GEMM on a pair of CTAs (tcgen05 cta_group::2), 2-bit slot format
+// and 1-bit g128, with the unpacked weights in tensor memory.
+//
+// y[m, n] = sum_k x'[m, k] * w[n, k],  w = s[n, k/128] * t[n, k]  (ternary
+// g128: news.ditty.ir, second paragraph).  The weights are the MMA's M side:
+// each thread unpacks its weight row into exact fp16 s*t (t is -1, 0 or +1 and
+// s an fp16 value) and writes it straight into tensor memory with tcgen05.st,
+// where the MMA reads it as operand A.  The tokens are the N side: x' tiles
+// come by TMA into shared memory as operand B.  So shared memory carries only
+// the x' tiles and the packed codes; the fp16 weights never touch it.
+//
+// One pair tile is 256 weight rows x BT tokens (BT = 128, 192 or 256, chosen
+// per shape for whole waves).  CTA r of the cluster owns weight rows 128 r .. 128 r + 127 (its
+// TMEM lanes) and loads tokens BT/2 r .. BT/2 r + BT/2 - 1 of the x' tile; one
+// M = 256 MMA issued by CTA 0 multiplies both CTAs' A (TMEM) by the B halves
+// of both CTAs, and each CTA's TMEM receives D for its own 128 weight rows and
+// all BT tokens.  Per K step of 16 a CTA's shared memory is read for BT/2
+// tokens only, half of what a one-CTA MMA of the same width reads.
+//
+// Warp roles in each CTA:
+//   warp 0     : TMA producer (x' half tile with 128B swizzle; packed codes);
+//   warp 1     : TMEM allocation for the pair; in CTA 0, the thread issuing
+//                the MMAs;
+//   warps 2-17 : unpack, four sets of four warps: warp w takes TMEM lanes
+//                32 (w % 4) .. + 31 and the stages kb = j, j + 4, ... of its
+//                set j = (w - 2) / 4, so each warp has four stages of MMA time
+//                for the fixed cost of one (barrier waits, the hand-off);
+//                then the epilogue (tcgen05.ld of D, convert, store y with
+//                the weight rows along the warp's lanes).
+// Hand-offs per stage s:
+//   full[s]  (each CTA): the CTA's x' half and codes landed (TMA);
+//   ready[s] (CTA 0)   : the 8 unpack warps of both CTAs wrote their A
+//                        slices and saw their x' half land (the other CTA's
+//                        warps arrive through the cluster's shared window);
+//   empty[s] (each CTA): the stage's MMAs are done (commit multicast to both
+//                        CTAs) - its x' half, codes and TMEM A slice are free.
+// The code order inside a 16-code chunk is the one the prep kernel writes x'
+// in (k = 0, 8, 1, 9, ..., 7, 15): the TMEM column j of a chunk holds the fp16
+// pair (w_j, w_{j+8}).
+//
+// Every wait is bounded; after a timeout a role stops waiting, records a fault
+// word and still reaches the final cluster barrier, so no CTA leaves while its
+// peer may touch its memory, and TMEM is always freed.
+#pragma once
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "gemv_tc.cuh"
+
+namespace tb {
+
+constexpr int kGpSets = 4;  // unpack warp sets (stage kb goes to set kb % 4)
+constexpr int kGpThreads = 32 * (2 + 4 * kGpSets);
+constexpr int kGpRows = 128;          // weight rows per CTA (TMEM lanes); 256 per pair
+constexpr int kGpPairRows = 2 * kGpRows;
+constexpr int kGpBK = 128;            // K per stage: one scale group, two 128-byte swizzle atoms of fp16
+constexpr int kGpAtomK = 64;          // K of one swizzle atom (128 bytes of fp16)
+constexpr int kGpASlots = kGpSets;    // TMEM A ring: set j owns slot j
+constexpr int kGpACols = kGpBK / 2;   // TMEM columns of a stage's A slice (2 fp16 a column)
+constexpr int kGpDCols = 256;         // D columns (tokens) at most; the A ring follows
+constexpr int kGpTmemCols = 512;
+constexpr int kGpSmemCap = 227 * 1024;
+static_assert(kGpDCols + kGpASlots * kGpACols <= kGpTmemCols, "TMEM budget");
+
+// x' half tile of a stage: two atoms of BT/2 rows x 128 bytes
+__host__ __device__ constexpr int gp_x_bytes(int bt) { return bt / 2 * kGpBK * 2; }
+// codes of a stage: 32 bytes a row (2-bit) or 16 (1-bit)
+__host__ __device__ constexpr int gp_w_row_bytes(int fmt) { return fmt == 0 ? kGpBK / 4 : kGpBK / 8; }
+__host__ __device__ constexpr int gp_stage_bytes(int bt, int fmt) {
+  return gp_x_bytes(bt) + kGpRows * gp_w_row_bytes(fmt);
+}
+// The shared-memory ring is deeper than the TMEM ring (copies run further
+// ahead than the unpack): as many stages as fit, at most 8.
+__host__ __device__ constexpr int gp_stages(int bt, int fmt) {
+  return (kGpSmemCap - 1024 - 256) / gp_stage_bytes(bt, fmt) < 8 ? (kGpSmemCap - 1024 - 256) / gp_stage_bytes(bt, fmt)
+                                                                   : 8;
+}
+__host__ __device__ constexpr int gp_smem_bytes(int bt, int fmt) {
+  return gp_stages(bt, fmt) * gp_stage_bytes(bt, fmt) + 1024 /*align*/ + 256 /*barriers*/;
+}
+// kind::f16, D fp32, A and B fp16 and K-major, N = bt tokens, M = 256 (pair).
+__host__ __device__ constexpr uint32_t gp_idesc(int bt) {
+  return (1u << 4) | (static_cast<uint32_t>(bt >> 3) << 17) | (static_cast<uint32_t>(kGpPairRows >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- cluster
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of both CTAs.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::
+          : "memory");
+}
+// Address of this CTA's shared variable at `saddr` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// Arrive on a barrier of either CTA of the cluster.  Default semantics
+// (release at CTA scope): measured on B200, the cluster-scope release form
+// held the arriving warp about 1600 cycles per arrival, once per stage.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// ---------------------------------------------------------------- tcgen05, pair forms
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (both CTAs' TMEM) += A (both CTAs' TMEM) x B (both CTAs' shared memory).
+__device__ __forceinline__ void umma_f16_pair_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrives on the barrier at this offset in both CTAs once the MMAs issued so
+// far complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+template <typename TOut>
+__device__ __forceinline__ void store_out(TOut* p, uint32_t v);
+template <>
+__device__ __forceinline__ void store_out<float>(float* p, uint32_t v) {
+  *p = __uint_as_float(v);
+}
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, uint32_t v) {
+  *p = __float2bfloat16_rn(__uint_as_float(v));
+}
+
+// 2-D tiled store of one box from shared memory (bulk group of this thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+// Named barrier `id` over `count` threads that also ANDs a predicate.
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+  asm volatile(
+      "cp.async.bulk.commit_group;\n\t"
+      "cp.async.bulk.wait_group.read 0;" ::
+          : "memory");
+}
+
+// kFmt: 0 = 2-bit slots, 2 = 1-bit g128.  tma_y: y goes out through shared
+// memory and one TMA store per CTA (rows 16-byte aligned), else by plain
+// stores.
+template <int BT, typename TOut, int kFmt>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                     const __grid_constant__ CUtensorMap tm_y, const GemmParams p, const int tma_y) {
+  static_assert(kFmt == 0 || kFmt == 2, "2-bit or 1-bit codes");
+  static_assert(BT % 64 == 0 && BT >= 128 && BT <= kGpDCols, "token tile");
+  constexpr int kX = gp_x_bytes(BT), kAtom = kX / 2, kW = kGpRows * gp_w_row_bytes(kFmt);
+  constexpr int kStage = gp_stage_bytes(BT, kFmt), S = gp_stages(BT, kFmt), SA = kGpASlots;
+  static_assert(kAtom % 1024 == 0 && kStage % 1024 == 0, "128B-swizzle atoms stay 1024-byte aligned");
+  static_assert(S >= SA, "the copies run at least as far ahead as the unpack");
+  static_assert(BT * kGpRows * static_cast<int>(sizeof(TOut)) <= S * kStage, "the y tile fits the stage ring");
+  constexpr uint32_t kIdesc = gp_idesc(BT);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kStage);  // copies landed
+  uint64_t* sfree = full + S;   // stage slot read: by the MMAs (x') and the unpack warps (codes)
+  uint64_t* ready = sfree + S;  // (CTA 0) A slot written and x' landed, in both CTAs
+  uint64_t* afree = ready + SA; // the MMAs reading an A slot are done
+  uint64_t* accum = afree + SA;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+
+  const uint32_t rank = cluster_rank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = static_cast<int>(blockIdx.x >> 1) * kGpPairRows + static_cast<int>(rank) * kGpRows;
+  const int m0 = blockIdx.y * BT;
+  const int nk = p.K / kGpBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sfree[s], 1 + 4);  // the MMAs' commit and the 4 warps of the stage's set
+    }
+    for (int a = 0; a < SA; ++a) {
+      mbar_init(&ready[a], 2 * 4);  // the 4 warps of the stage's set in each CTA
+      mbar_init(&afree[a], 1);
+    }
+    mbar_init(accum, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kGpTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  const uint32_t tmem_a = tmem_d + kGpDCols;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      prefetch_tensormap(&tm_x);
+      prefetch_tensormap(&tm_w);
+      pdl_wait();  // x' comes from the prep kernel
+      const bool stall = test_stall_copies();  // failure-detection test: no copies
+      int issued = 0;
+      for (int kb = 0; kb < nk && !stall; ++kb) {
+        const int s = kb % S;
+        if (kb >= S && !mbar_wait(&sfree[s], ((kb / S) & 1) ^ 1, FAULT_WAIT_EMPTY)) break;
+        uint8_t* st = smem + s * kStage;
+        mbar_arrive_expect_tx(&full[s], kX + kW);
+        const int my = m0 + static_cast<int>(rank) * (BT / 2);
+        tma_load_2d(st, &tm_x, kb * kGpBK, my, &full[s]);
+        tma_load_2d(st + kAtom, &tm_x, kb * kGpBK + kGpAtomK, my, &full[s]);
+        // x in 32-bit words: 8 words a stage (2-bit), 4 (1-bit)
+        tma_load_2d(st + kX, &tm_w, kb * (kW / kGpRows / 4), n0, &full[s]);
+        issued = kb + 1;
+      }
+      // the last copies issued land before the CTA may leave
+      for (int kb = issued > S ? issued - S : 0; kb < issued; ++kb)
+        if (!mbar_wait(&full[kb % S], (kb / S) & 1, FAULT_WAIT_FULL)) break;
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA (CTA 0)
+    if (rank == 0 && lane == 0) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % S, a = kb % SA;
+        if (!mbar_wait(&ready[a], (kb / SA) & 1, FAULT_WAIT_FULL)) break;
+        tc_fence_after();
+        const uint32_t b = smem_u32(smem + s * kStage);
+#pragma unroll
+        for (int kk = 0; kk < kGpBK / 16; ++kk)
+          umma_f16_pair_ts(tmem_d, tmem_a + static_cast<uint32_t>(a * kGpACols + 8 * kk),
+                           umma_desc_sw128(b + (kk >> 2) * kAtom + 32 * (kk & 3)), kIdesc,
+                           (kb | kk) != 0 ? 1u : 0u);
+        umma_commit_pair(&sfree[s]);
+        umma_commit_pair(&afree[a]);
+      }
+      umma_commit_pair(accum);
+    }
+  } else {
+    // ---------------------------------------------------------------- unpack
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int set = (warp - 2) >> 2;   // stages set, set + 4, ... (A slot set)
+    const int r = 32 * q + lane;       // weight row of this CTA = TMEM lane
+    const int n = n0 + r;
+    const bool row_ok = n < p.N;
+    const int G = p.K / 128;
+    const uint16_t* srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
+    const __half2 k1024 = __float2half2_rn(1024.f);
+    const __half2 k1 = __float2half2_rn(1.f);
+    const __half2 kinv256 = __float2half2_rn(1.f / 256.f);
+    const __half2 km4 = __float2half2_rn(-4.f);
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+    const uint32_t ta = tmem_a + lane_addr + static_cast<uint32_t>(set * kGpACols);
+    const uint32_t ready0 = cluster_map(smem_u32(&ready[set]), 0);  // CTA 0's ready barrier of this set
+    uint16_t s_bits = (row_ok && set < nk) ? srow[set] : uint16_t(0);  // stage kb is scale group kb
+    for (int kb = set; kb < nk; kb += kGpSets) {
+      const int s = kb % S;
+      const int kn = kb + kGpSets;  // this warp's next stage: its scale is loaded a stage early
+      const uint16_t s_nb = (row_ok && kn < nk) ? srow[kn] : uint16_t(0);
+      // every lane waits (each reads the stage); the warp leaves together
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (kb / S) & 1, FAULT_WAIT_FULL))) break;
+      const uint8_t* wrow = smem + s * kStage + kX + r * gp_w_row_bytes(kFmt);
+      uint4 wv[2];
+      wv[0] = *reinterpret_cast<const uint4*>(wrow);
+      wv[1] = kFmt == 0 ? *reinterpret_cast<const uint4*>(wrow + 16) : make_uint4(0, 0, 0, 0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sfree[s]);  // the codes are in registers
+      // the MMAs of stage kb - 4 are done with this A slot
+      if (kb >= SA && !__all_sync(0xffffffffu, mbar_wait(&afree[set], ((kb / SA) & 1) ^ 1, FAULT_WAIT_MMA)))
+        break;
+      tc_fence_after();
+      const __half sc = __ushort_as_half(s_bits);
+      const __half2 s2 = __halves2half2(sc, sc);
+      const __half2 ns2 = __hneg2(s2);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // codes 64 half .. 64 half + 63 -> 32 TMEM columns
+        uint32_t o[32];
+        if constexpr (kFmt == 2) {
+          // chunk c of the 128 codes (16 codes) is half c & 1 of word c >> 1.
+          // z holds the chunk's low 8 codes in bits 0-7 and its high 8 in bits
+          // 16-23; (z << (15 - j)) & 0x80008000 puts codes j and j + 8 on the
+          // sign bits of a half2, and XOR with (-s, -s) gives (s t_j, s t_{j+8}).
+          const uint32_t nb = *reinterpret_cast<const uint32_t*>(&ns2);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t w = (&wv[0].x)[2 * half + (c >> 1)];
+            const uint32_t z = __byte_perm(w, 0u, (c & 1) ? 0x4342u : 0x4140u);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) o[8 * c + j] = ((z << (15 - j)) & 0x80008000u) ^ nb;
+          }
+        } else {
+#pragma unroll
+          for (int wd = 0; wd < 4; ++wd) {
+            const uint32_t w = (&wv[half].x)[wd];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t ws = w >> (2 * j);
+              const uint32_t lo = (ws & 0x00030003u) | 0x64006400u;  // 1024 + c_j, 1024 + c_{j+8}
+              const uint32_t hi = (ws & 0x03000300u) | 0x64006400u;  // 1024 + 256 c_{j+4}, ...
+              const __half2 clo = __hfma2(*reinterpret_cast<const __half2*>(&lo), k1, __hneg2(k1024));
+              const __half2 chi = __hfma2(*reinterpret_cast<const __half2*>(&hi), kinv256, km4);
+              const __half2 vlo = __hfma2(clo, s2, ns2);
+              const __half2 vhi = __hfma2(chi, s2, ns2);
+              o[8 * wd + j] = *reinterpret_cast<const uint32_t*>(&vlo);
+              o[8 * wd + j + 4] = *reinterpret_cast<const uint32_t*>(&vhi);
+            }
+          }
+        }
+        tmem_st32(ta + static_cast<uint32_t>(32 * half), o);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(ready0);
+      s_bits = s_nb;
+    }
+    // ---------------------------------------------------------------- epilogue
+    constexpr int kEpiThreads = 4 * kGpSets * 32;
+    // one decision for all epilogue warps (they meet at a named barrier below)
+    if (bar_and(1, kEpiThreads, mbar_wait(accum, 0, FAULT_WAIT_EPILOGUE))) {
+      tc_fence_after();
+      constexpr int kCols = BT / kGpSets;  // tokens of this warp: set * kCols .. + kCols - 1
+      if (tma_y) {
+        // y tile [BT tokens][128 rows] in the (now idle) stage ring, then one
+        // TMA store, which also drops what lies beyond M or N
+        TOut* ty = reinterpret_cast<TOut*>(smem);
+#pragma unroll 1
+        for (int c0 = set * kCols; c0 < (set + 1) * kCols; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_cols<16>(tmem_d + lane_addr + static_cast<uint32_t>(c0), v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) store_out<TOut>(ty + (c0 + j) * kGpRows + r, v[j]);
+        }
+        fence_proxy_async_shared();  // generic-proxy stores -> visible to the TMA store
+        asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+        if (warp == 2 && lane == 0 && n0 < p.N) {  // a CTA past the last row has nothing to store
+          tma_store_2d(&tm_y, ty, n0, m0);
+          bulk_commit_and_wait_read();
+        }
+      } else {
+        TOut* y = reinterpret_cast<TOut*>(p.y) + n;
+#pragma unroll 1
+        for (int c0 = set * kCols; c0 < (set + 1) * kCols; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_cols<16>(tmem_d + lane_addr + static_cast<uint32_t>(c0), v);
+          tmem_ld_wait();
+          const int mb = m0 + c0;
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (mb + j < p.M) store_out<TOut>(y + static_cast<int64_t>(mb + j) * p.N, v[j]);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();  // neither CTA leaves while its peer may still touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_d, kGpTmemCols);
+  }
+}
+
+}  // namespace tb

@@ -48,23 +48,28 @@ constexpr int kGemmSmemCap = 227 * 1024;  // dynamic shared memory of one CTA at
 constexpr int kGemmUnpackWarps = 8;
 constexpr int kGemmThreads = 32 * (2 + kGemmUnpackWarps);
 constexpr int kGemmTmemCols = 512;
-// per tile (BM tokens, BN weight rows): A (fp16 x'), B (fp16 s*t) and the
-// packed codes of a stage
+// per tile (BM tokens, BN weight rows): A (fp16 x') and the packed codes of a
+// stage come by TMA into a ring of stages; B (fp16 s*t, written by the unpack
+// warps) has a ring of its own of kGemmBSlots buffers, so the copies run as
+// far ahead as the stage ring allows while the unpack works one stage ahead of
+// the MMAs.
+constexpr int kGemmBSlots = 2;
 __host__ __device__ constexpr int gemm_a_bytes(int bm) { return bm * kGemmBK * 2; }
 __host__ __device__ constexpr int gemm_b_bytes(int bn) { return bn * kGemmBK * 2; }
 __host__ __device__ constexpr int gemm_w_bytes(int bn) { return bn * kGemmBK / 4; }
 __host__ __device__ constexpr int gemm_stage_bytes(int bm, int bn) {
-  return gemm_a_bytes(bm) + gemm_b_bytes(bn) + gemm_w_bytes(bn);
+  return gemm_a_bytes(bm) + gemm_w_bytes(bn);
 }
 // As many stages as fit (at most 8): small tiles have little MMA work per
 // stage, so more stages are in flight to cover the copies' latency.
 __host__ __device__ constexpr int gemm_stages(int bm, int bn) {
-  return (kGemmSmemCap - 1024 - 256) / gemm_stage_bytes(bm, bn) < 8
-             ? (kGemmSmemCap - 1024 - 256) / gemm_stage_bytes(bm, bn)
+  return (kGemmSmemCap - 1024 - 256 - kGemmBSlots * gemm_b_bytes(bn)) / gemm_stage_bytes(bm, bn) < 8
+             ? (kGemmSmemCap - 1024 - 256 - kGemmBSlots * gemm_b_bytes(bn)) / gemm_stage_bytes(bm, bn)
              : 8;
 }
 __host__ __device__ constexpr int gemm_smem_bytes(int bm, int bn) {
-  return gemm_stages(bm, bn) * gemm_stage_bytes(bm, bn) + 1024 /*align*/ + 256 /*barriers*/;
+  return gemm_stages(bm, bn) * gemm_stage_bytes(bm, bn) + kGemmBSlots * gemm_b_bytes(bn) + 1024 /*align*/ +
+         256 /*barriers*/;
 }
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B fp16
@@ -224,10 +229,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr uint32_t kIdesc = gemm_idesc(BN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmStages * kStage);
-  uint64_t* bready = full + kGemmStages;
-  uint64_t* empty = bready + kGemmStages;
-  uint64_t* accum = empty + kGemmStages;
+  uint8_t* bring = smem + kGemmStages * kStage;  // kGemmBSlots x kB, 1 KB aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(bring + kGemmBSlots * kB);
+  uint64_t* empty = full + kGemmStages;
+  uint64_t* bfull = empty + kGemmStages;
+  uint64_t* bempty = bfull + kGemmBSlots;
+  uint64_t* accum = bempty + kGemmBSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,8 +244,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&bready[s], kGemmUnpackWarps);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + kGemmUnpackWarps);  // the MMAs read A, the unpack warps read the codes
+    }
+    for (int b = 0; b < kGemmBSlots; ++b) {
+      mbar_init(&bfull[b], kGemmUnpackWarps);
+      mbar_init(&bempty[b], 1);
     }
     mbar_init(accum, 1);
     fence_mbar_init();
@@ -269,7 +279,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_arrive_expect_tx(&full[s], kA + (wload ? kW : 0));
         tma_load_2d(st, &tm_x, kb * kGemmBK, m0, &full[s]);
         // x in 32-bit words: 2-bit, 4 words per stage; 1-bit, 4 words per two stages
-        if (wload) tma_load_2d(st + kA + kB, &tm_w, kFmt == 0 ? kb * 4 : (kb >> 1) * 4, n0, &full[s]);
+        if (wload) tma_load_2d(st + kA, &tm_w, kFmt == 0 ? kb * 4 : (kb >> 1) * 4, n0, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -277,13 +287,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       bool ok = true;
       for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % kGemmStages;
+        const int s = kb % kGemmStages, bs = kb % kGemmBSlots;
         const uint32_t par = (kb / kGemmStages) & 1;
-        ok = mbar_wait(&full[s], par, FAULT_WAIT_FULL) && mbar_wait(&bready[s], par, FAULT_WAIT_FULL);
+        ok = mbar_wait(&full[s], par, FAULT_WAIT_FULL) &&
+             mbar_wait(&bfull[bs], (kb / kGemmBSlots) & 1, FAULT_WAIT_FULL);
         if (!ok) break;
         tc_fence_after();
         const uint32_t a = smem_u32(smem + s * kStage);
-        const uint32_t b = a + kA;
+        const uint32_t b = smem_u32(bring + bs * kB);
 #pragma unroll
         for (int kk = 0; kk < kGemmBK / 16; ++kk) {
           const uint64_t bd = umma_desc_sw128(b + 32 * kk);
@@ -293,6 +304,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             umma_f16(tmem + BN, umma_desc_sw128(a + kGemmUM * 128 + 32 * kk), bd, kIdesc, acc);
         }
         umma_commit(&empty[s]);
+        umma_commit(&bempty[bs]);
       }
       umma_commit(accum);
     }
@@ -314,7 +326,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t wcur[2] = {0u, 0u}, wnext[2] = {0u, 0u};  // 1-bit codes of this and the next stage
     bool ok = true;
     for (int kb = 0; kb < nk && ok; ++kb) {
-      const int s = kb % kGemmStages;
+      const int s = kb % kGemmStages, bs = kb % kGemmBSlots;
       if (!mbar_wait(&full[s], (kb / kGemmStages) & 1, FAULT_WAIT_FULL)) {
         ok = false;
         break;
@@ -325,16 +337,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (g + 1 < G) s_next = __ushort_as_half(row_ok ? srow[g + 1] : uint16_t(0));
       }
       uint8_t* st = smem + s * kStage;
+      // this stage's codes into registers; then the stage's slot is free as
+      // far as the unpack is concerned
+      uint4 w4 = make_uint4(0, 0, 0, 0);
+      if (in_tile && (kFmt == 0 || (kb & 1) == 0)) w4 = *reinterpret_cast<const uint4*>(st + kA + r * 16);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      // the MMAs of stage kb - kGemmBSlots are done with this B buffer
+      if (kb >= kGemmBSlots && !mbar_wait(&bempty[bs], ((kb / kGemmBSlots) & 1) ^ 1, FAULT_WAIT_EMPTY)) {
+        ok = false;
+        break;
+      }
       const __half2 s2 = __halves2half2(s_cur, s_cur);
       const __half2 ns2 = __hneg2(s2);
-      uint8_t* row = st + kA + r * 128;
+      uint8_t* row = bring + bs * kB + r * 128;
       if constexpr (kFmt == 2) {
         // 1-bit: 16-code chunk c of the stage (c = 0..3) is half c & 1 of
         // word c >> 1.  z holds its low 8 codes in bits 0-7 and its high 8 in
         // bits 16-23; (z << (15 - j)) & 0x80008000 puts codes j and j + 8 on
         // the sign bits of a half2, and XOR with (-s, -s) gives (s t_j, s t_{j+8}).
         if ((kb & 1) == 0 && in_tile) {
-          const uint4 w4 = *reinterpret_cast<const uint4*>(st + kA + kB + r * 16);
           wcur[0] = w4.x;
           wcur[1] = w4.y;
           wnext[0] = w4.z;
@@ -354,8 +376,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           *reinterpret_cast<uint4*>(row + 16 * ((2 * c + 1) ^ sw)) = make_uint4(o[4], o[5], o[6], o[7]);
         }
       }
-      const uint4 w4 = (kFmt == 0 && in_tile) ? *reinterpret_cast<const uint4*>(st + kA + kB + r * 16)
-                                              : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int wd = 0; wd < 4 && in_tile && kFmt == 0; ++wd) {
         const uint32_t w = (&w4.x)[wd];
@@ -377,7 +397,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       fence_proxy_async_shared();  // generic-proxy stores -> visible to the tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bready[s]);
+      if (lane == 0) mbar_arrive(&bfull[bs]);
     }
     // ---------------------------------------------------------------- epilogue
     if (mbar_wait(accum, 0, FAULT_WAIT_EPILOGUE)) {

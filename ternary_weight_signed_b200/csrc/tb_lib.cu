@@ -15,6 +15,7 @@
 #include "tb_device.cuh"
 
 #include "gemm_tc.cuh"
+#include "gemm_pair.cuh"
 #include "gemm_i8.cuh"
 #include "gemv.cuh"
 #include "gemv_m1.cuh"
@@ -958,52 +959,57 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
     default: launch_prep_gemm<float>(a, xh); break;
   }
   if (launch_status() != TB_OK) return TB_ERR_CUDA;
-  int bm = 256, bn = 256;
-  gemm_tiles(a.M, a.N, d->sm_count, &bm, &bn);
-  const int64_t mt = (a.M + bm - 1) / bm;
+  // token tile: 256, or 128 up to 128 tokens.  Measured on B200, a pair
+  // MMA with A in TMEM takes about 130 cycles at N = 128 and at N = 256 alike
+  // (148 at N = 192), so narrower tiles only pay where the tokens are few.
+  const int64_t pairs_n = (a.N + kGpPairRows - 1) / kGpPairRows;
+  const int bt = a.M <= 128 ? 128 : 256;
   CUtensorMap tm_x, tm_w;
-  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGemmBK,
-                  static_cast<uint32_t>(bm), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGpAtomK,
+                  static_cast<uint32_t>(bt / 2), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
-  // 16 bytes of a row per box: 64 codes (2-bit, one stage) or 128 codes (1-bit, two stages)
+  // the 128 codes of a stage: 32 bytes of a row (2-bit) or 16 (1-bit)
   const uint64_t wrow = one_bit ? a.K / 8 : a.K / 4;
-  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, wrow / 4, a.N, wrow, 4,
-                  static_cast<uint32_t>(bn)) != TB_OK)
+  if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, wrow / 4, a.N, wrow,
+                  static_cast<uint32_t>(gp_w_row_bytes(one_bit ? 2 : 0) / 4), static_cast<uint32_t>(kGpRows)) != TB_OK)
     return TB_ERR_CUDA;
+  // y leaves through one TMA store per CTA where its rows are 16-byte aligned
+  const int ysz = a.yt == TB_FP32 ? 4 : 2;
+  CUtensorMap tm_y = tm_x;
+  int tma_y = 0;
+  if (aligned(a.y, 16) && (a.N * ysz) % 16 == 0) {
+    if (make_map_2d(&tm_y, a.yt == TB_FP32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ysz,
+                    a.y, a.N, a.M, a.N * ysz, static_cast<uint32_t>(kGpRows), static_cast<uint32_t>(bt)) != TB_OK)
+      return TB_ERR_CUDA;
+    tma_y = 1;
+  }
   GemmParams gp;
   gp.M = static_cast<int>(a.M);
   gp.N = static_cast<int>(a.N);
   gp.K = static_cast<int>(a.K);
   gp.y = a.y;
   gp.scales = a.scales;
-  const dim3 grid(static_cast<unsigned>((a.N + bn - 1) / bn), static_cast<unsigned>(mt));
-#define TB_GEMM_LAUNCH_F(BM, BN, F)                                                                         \
-  {                                                                                                          \
-    if (a.yt == TB_FP32) {                                                                                   \
-      auto k = gemm_tc_kernel<BM, BN, float, F>;                                                             \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
-      return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BM, BN)), a.st, tm_x, \
-                        tm_w, gp);                                                                           \
-    }                                                                                                        \
-    auto k = gemm_tc_kernel<BM, BN, __nv_bfloat16, F>;                                                       \
-    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                       \
-    return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gemm_smem_bytes(BM, BN)), a.st, tm_x,   \
-                      tm_w, gp);                                                                             \
+  const dim3 grid(static_cast<unsigned>(2 * pairs_n), static_cast<unsigned>((a.M + bt - 1) / bt));
+#define TB_GP_LAUNCH(BT, F)                                                                               \
+  {                                                                                                       \
+    if (a.yt == TB_FP32) {                                                                                \
+      auto k = gemm_pair_kernel<BT, float, F>;                                                            \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                  \
+      return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F)), a.st, tm_x, \
+                        tm_w, tm_y, gp, tma_y);                                                           \
+    }                                                                                                     \
+    auto k = gemm_pair_kernel<BT, __nv_bfloat16, F>;                                                      \
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                    \
+    return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F)), a.st, tm_x,   \
+                      tm_w, tm_y, gp, tma_y);                                                             \
   }
-#define TB_GEMM_LAUNCH(BM, BN)               \
-  if (bm == BM && bn == BN) {                \
-    if (one_bit) TB_GEMM_LAUNCH_F(BM, BN, 2) \
-    TB_GEMM_LAUNCH_F(BM, BN, 0)              \
+  if (bt == 128) {
+    if (one_bit) TB_GP_LAUNCH(128, 2)
+    TB_GP_LAUNCH(128, 0)
   }
-  TB_GEMM_LAUNCH(256, 256)
-  TB_GEMM_LAUNCH(256, 192)
-  TB_GEMM_LAUNCH(256, 128)
-  TB_GEMM_LAUNCH(128, 256)
-  TB_GEMM_LAUNCH(128, 192)
-  TB_GEMM_LAUNCH(128, 128)
-#undef TB_GEMM_LAUNCH
-#undef TB_GEMM_LAUNCH_F
-  return TB_ERR_SHAPE;
+  if (one_bit) TB_GP_LAUNCH(256, 2)
+  TB_GP_LAUNCH(256, 0)
+#undef TB_GP_LAUNCH
 }
 
 // ------------------------------------------------------------------ linear: integer-mode GEMM
