@@ -42,6 +42,7 @@
 // word and still reaches the final cluster barrier, so no CTA leaves while its
 // peer may touch its memory, and TMEM is always freed.
 #pragma once
+#include "gemm_i8.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
@@ -52,34 +53,44 @@ constexpr int kGpSets = 4;  // unpack warp sets (stage kb goes to set kb % 4)
 constexpr int kGpThreads = 32 * (2 + 4 * kGpSets);
 constexpr int kGpRows = 128;          // weight rows per CTA (TMEM lanes); 256 per pair
 constexpr int kGpPairRows = 2 * kGpRows;
-constexpr int kGpBK = 128;            // K per stage: one scale group, two 128-byte swizzle atoms of fp16
-constexpr int kGpAtomK = 64;          // K of one swizzle atom (128 bytes of fp16)
+// A stage is two 128-byte swizzle atoms of x along K: 128 fp16 values (one
+// scale group) or 256 int8 values; either way 64 TMEM columns of A and eight
+// MMAs (K = 16 for kind::f16, 32 for kind::i8).
+__host__ __device__ constexpr int gp_bk(bool integer) { return integer ? 256 : 128; }
+__host__ __device__ constexpr int gp_atom_k(bool integer) { return gp_bk(integer) / 2; }
+constexpr int kGpAtomBytes = 128;
 constexpr int kGpASlots = kGpSets;    // TMEM A ring: set j owns slot j
-constexpr int kGpACols = kGpBK / 2;   // TMEM columns of a stage's A slice (2 fp16 a column)
+constexpr int kGpACols = 64;          // TMEM columns of a stage's A slice
 constexpr int kGpDCols = 256;         // D columns (tokens) at most; the A ring follows
 constexpr int kGpTmemCols = 512;
 constexpr int kGpSmemCap = 227 * 1024;
 static_assert(kGpDCols + kGpASlots * kGpACols <= kGpTmemCols, "TMEM budget");
 
-// x' half tile of a stage: two atoms of BT/2 rows x 128 bytes
-__host__ __device__ constexpr int gp_x_bytes(int bt) { return bt / 2 * kGpBK * 2; }
-// codes of a stage: 32 bytes a row (2-bit) or 16 (1-bit)
-__host__ __device__ constexpr int gp_w_row_bytes(int fmt) { return fmt == 0 ? kGpBK / 4 : kGpBK / 8; }
-__host__ __device__ constexpr int gp_stage_bytes(int bt, int fmt) {
-  return gp_x_bytes(bt) + kGpRows * gp_w_row_bytes(fmt);
+// x half tile of a stage: two atoms of BT/2 rows x 128 bytes
+__host__ __device__ constexpr int gp_x_bytes(int bt) { return bt / 2 * 2 * kGpAtomBytes; }
+// codes of a stage per row: 2 bits (fmt 0) or 1 bit (fmt 2) a code
+__host__ __device__ constexpr int gp_w_row_bytes(int fmt, bool integer) {
+  return fmt == 0 ? gp_bk(integer) / 4 : gp_bk(integer) / 8;
+}
+__host__ __device__ constexpr int gp_stage_bytes(int bt, int fmt, bool integer) {
+  return gp_x_bytes(bt) + kGpRows * gp_w_row_bytes(fmt, integer);
 }
 // The shared-memory ring is deeper than the TMEM ring (copies run further
 // ahead than the unpack): as many stages as fit, at most 8.
-__host__ __device__ constexpr int gp_stages(int bt, int fmt) {
-  return (kGpSmemCap - 1024 - 256) / gp_stage_bytes(bt, fmt) < 8 ? (kGpSmemCap - 1024 - 256) / gp_stage_bytes(bt, fmt)
-                                                                   : 8;
+__host__ __device__ constexpr int gp_stages(int bt, int fmt, bool integer) {
+  return (kGpSmemCap - 1024 - 256) / gp_stage_bytes(bt, fmt, integer) < 8
+             ? (kGpSmemCap - 1024 - 256) / gp_stage_bytes(bt, fmt, integer)
+             : 8;
 }
-__host__ __device__ constexpr int gp_smem_bytes(int bt, int fmt) {
-  return gp_stages(bt, fmt) * gp_stage_bytes(bt, fmt) + 1024 /*align*/ + 256 /*barriers*/;
+__host__ __device__ constexpr int gp_smem_bytes(int bt, int fmt, bool integer) {
+  return gp_stages(bt, fmt, integer) * gp_stage_bytes(bt, fmt, integer) + 1024 /*align*/ + 256 /*barriers*/;
 }
-// kind::f16, D fp32, A and B fp16 and K-major, N = bt tokens, M = 256 (pair).
-__host__ __device__ constexpr uint32_t gp_idesc(int bt) {
-  return (1u << 4) | (static_cast<uint32_t>(bt >> 3) << 17) | (static_cast<uint32_t>(kGpPairRows >> 4) << 24);
+// Instruction descriptor, M = 256 (pair), N = bt tokens, both operands
+// K-major.  kind::f16: D fp32 (bits 4-5 = 1), A and B fp16.  kind::i8: D s32
+// (bits 4-5 = 2), A and B signed 8-bit (bits 7 and 10).
+__host__ __device__ constexpr uint32_t gp_idesc(int bt, bool integer) {
+  return (integer ? (2u << 4) | (1u << 7) | (1u << 10) : (1u << 4)) | (static_cast<uint32_t>(bt >> 3) << 17) |
+         (static_cast<uint32_t>(kGpPairRows >> 4) << 24);
 }
 
 // ---------------------------------------------------------------- cluster
@@ -120,13 +131,21 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 // D (both CTAs' TMEM) += A (both CTAs' TMEM) x B (both CTAs' shared memory).
-__device__ __forceinline__ void umma_f16_pair_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+template <bool kInt>
+__device__ __forceinline__ void umma_pair_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  if constexpr (kInt)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 // Arrives on the barrier at this offset in both CTAs once the MMAs issued so
 // far complete.
@@ -146,6 +165,10 @@ __device__ __forceinline__ void store_out<float>(float* p, uint32_t v) {
 template <>
 __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, uint32_t v) {
   *p = __float2bfloat16_rn(__uint_as_float(v));
+}
+template <>
+__device__ __forceinline__ void store_out<int32_t>(int32_t* p, uint32_t v) {
+  *p = static_cast<int32_t>(v);
 }
 
 // 2-D tiled store of one box from shared memory (bulk group of this thread).
@@ -174,21 +197,23 @@ __device__ __forceinline__ void bulk_commit_and_wait_read() {
           : "memory");
 }
 
-// kFmt: 0 = 2-bit slots, 2 = 1-bit g128.  tma_y: y goes out through shared
-// memory and one TMA store per CTA (rows 16-byte aligned), else by plain
-// stores.
-template <int BT, typename TOut, int kFmt>
+// kFmt: 0 = 2-bit slots, 2 = 1-bit g128.  kInt: integer mode (int8 x, no
+// rotation, no scales, exact int32 y; A = t as signed bytes), else fp16 x' and
+// A = fp16(s t).  tma_y: y goes out through shared memory and one TMA store
+// per CTA (rows 16-byte aligned), else by plain stores.
+template <int BT, typename TOut, int kFmt, bool kInt>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_y, const GemmParams p, const int tma_y) {
   static_assert(kFmt == 0 || kFmt == 2, "2-bit or 1-bit codes");
   static_assert(BT % 64 == 0 && BT >= 128 && BT <= kGpDCols, "token tile");
-  constexpr int kX = gp_x_bytes(BT), kAtom = kX / 2, kW = kGpRows * gp_w_row_bytes(kFmt);
-  constexpr int kStage = gp_stage_bytes(BT, kFmt), S = gp_stages(BT, kFmt), SA = kGpASlots;
+  constexpr int kBK = gp_bk(kInt), kAtomK = gp_atom_k(kInt), kWr = gp_w_row_bytes(kFmt, kInt);
+  constexpr int kX = gp_x_bytes(BT), kAtom = kX / 2, kW = kGpRows * kWr;
+  constexpr int kStage = gp_stage_bytes(BT, kFmt, kInt), S = gp_stages(BT, kFmt, kInt), SA = kGpASlots;
   static_assert(kAtom % 1024 == 0 && kStage % 1024 == 0, "128B-swizzle atoms stay 1024-byte aligned");
   static_assert(S >= SA, "the copies run at least as far ahead as the unpack");
   static_assert(BT * kGpRows * static_cast<int>(sizeof(TOut)) <= S * kStage, "the y tile fits the stage ring");
-  constexpr uint32_t kIdesc = gp_idesc(BT);
+  constexpr uint32_t kIdesc = gp_idesc(BT, kInt);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kStage);  // copies landed
@@ -202,7 +227,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = static_cast<int>(blockIdx.x >> 1) * kGpPairRows + static_cast<int>(rank) * kGpRows;
   const int m0 = blockIdx.y * BT;
-  const int nk = p.K / kGpBK;
+  // integer mode: K a multiple of 128; a last half stage reads zeros past K
+  const int nk = (p.K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -240,10 +266,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
         uint8_t* st = smem + s * kStage;
         mbar_arrive_expect_tx(&full[s], kX + kW);
         const int my = m0 + static_cast<int>(rank) * (BT / 2);
-        tma_load_2d(st, &tm_x, kb * kGpBK, my, &full[s]);
-        tma_load_2d(st + kAtom, &tm_x, kb * kGpBK + kGpAtomK, my, &full[s]);
-        // x in 32-bit words: 8 words a stage (2-bit), 4 (1-bit)
-        tma_load_2d(st + kX, &tm_w, kb * (kW / kGpRows / 4), n0, &full[s]);
+        tma_load_2d(st, &tm_x, kb * kBK, my, &full[s]);
+        tma_load_2d(st + kAtom, &tm_x, kb * kBK + kAtomK, my, &full[s]);
+        // x in 32-bit words: the codes of a stage are kWr bytes of each row
+        tma_load_2d(st + kX, &tm_w, kb * (kWr / 4), n0, &full[s]);
         issued = kb + 1;
       }
       // the last copies issued land before the CTA may leave
@@ -259,8 +285,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
         tc_fence_after();
         const uint32_t b = smem_u32(smem + s * kStage);
 #pragma unroll
-        for (int kk = 0; kk < kGpBK / 16; ++kk)
-          umma_f16_pair_ts(tmem_d, tmem_a + static_cast<uint32_t>(a * kGpACols + 8 * kk),
+        for (int kk = 0; kk < 8; ++kk)
+          umma_pair_ts<kInt>(tmem_d, tmem_a + static_cast<uint32_t>(a * kGpACols + 8 * kk),
                            umma_desc_sw128(b + (kk >> 2) * kAtom + 32 * (kk & 3)), kIdesc,
                            (kb | kk) != 0 ? 1u : 0u);
         umma_commit_pair(&sfree[s]);
@@ -276,7 +302,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
     const int n = n0 + r;
     const bool row_ok = n < p.N;
     const int G = p.K / 128;
-    const uint16_t* srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
+    const bool scaled = !kInt && row_ok;  // integer mode has no scales
+    const uint16_t* srow = kInt ? nullptr : p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
     const __half2 k1024 = __float2half2_rn(1024.f);
     const __half2 k1 = __float2half2_rn(1.f);
     const __half2 kinv256 = __float2half2_rn(1.f / 256.f);
@@ -284,17 +311,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     const uint32_t ta = tmem_a + lane_addr + static_cast<uint32_t>(set * kGpACols);
     const uint32_t ready0 = cluster_map(smem_u32(&ready[set]), 0);  // CTA 0's ready barrier of this set
-    uint16_t s_bits = (row_ok && set < nk) ? srow[set] : uint16_t(0);  // stage kb is scale group kb
+    uint16_t s_bits = (scaled && set < nk) ? srow[set] : uint16_t(0);  // fp16: stage kb is scale group kb
     for (int kb = set; kb < nk; kb += kGpSets) {
       const int s = kb % S;
       const int kn = kb + kGpSets;  // this warp's next stage: its scale is loaded a stage early
-      const uint16_t s_nb = (row_ok && kn < nk) ? srow[kn] : uint16_t(0);
+      const uint16_t s_nb = (scaled && kn < nk) ? srow[kn] : uint16_t(0);
       // every lane waits (each reads the stage); the warp leaves together
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (kb / S) & 1, FAULT_WAIT_FULL))) break;
-      const uint8_t* wrow = smem + s * kStage + kX + r * gp_w_row_bytes(kFmt);
-      uint4 wv[2];
-      wv[0] = *reinterpret_cast<const uint4*>(wrow);
-      wv[1] = kFmt == 0 ? *reinterpret_cast<const uint4*>(wrow + 16) : make_uint4(0, 0, 0, 0);
+      const uint8_t* wrow = smem + s * kStage + kX + r * kWr;
+      uint4 wv[kWr / 16];
+#pragma unroll
+      for (int i = 0; i < kWr / 16; ++i) wv[i] = *reinterpret_cast<const uint4*>(wrow + 16 * i);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sfree[s]);  // the codes are in registers
       // the MMAs of stage kb - 4 are done with this A slot
@@ -307,7 +334,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {  // codes 64 half .. 64 half + 63 -> 32 TMEM columns
         uint32_t o[32];
-        if constexpr (kFmt == 2) {
+        if constexpr (kInt && kFmt == 0) {
+          // codes 128 half .. + 127: packed words 8 half .. + 7, each as 16
+          // bytes c = t + 1 in natural order, then t = c - 1 bytewise:
+          // (c + 0x7F) ^ 0x80 never carries out of a byte (c <= 2)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 c4 = gi8_codes16((&wv[0].x)[8 * half + i]);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) o[4 * i + b] = ((&c4.x)[b] + 0x7F7F7F7Fu) ^ 0x80808080u;
+          }
+        } else if constexpr (kInt) {
+          // 1-bit: codes 128 half .. + 127 are words 4 half .. + 3, 32 codes a
+          // word; t = 2 b - 1 bytewise as (2 b + 0x7F) ^ 0x80
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t w = (&wv[0].x)[4 * half + i];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) o[8 * i + rr] = ((gi8_bits4(w, rr) << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
+          }
+        } else if constexpr (kFmt == 2) {
           // chunk c of the 128 codes (16 codes) is half c & 1 of word c >> 1.
           // z holds the chunk's low 8 codes in bits 0-7 and its high 8 in bits
           // 16-23; (z << (15 - j)) & 0x80008000 puts codes j and j + 8 on the

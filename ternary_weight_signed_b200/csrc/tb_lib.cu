@@ -965,13 +965,14 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   const int64_t pairs_n = (a.N + kGpPairRows - 1) / kGpPairRows;
   const int bt = a.M <= 128 ? 128 : 256;
   CUtensorMap tm_x, tm_w;
-  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, kGpAtomK,
+  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, a.K, a.M, a.K * 2, gp_atom_k(false),
                   static_cast<uint32_t>(bt / 2), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
   // the 128 codes of a stage: 32 bytes of a row (2-bit) or 16 (1-bit)
   const uint64_t wrow = one_bit ? a.K / 8 : a.K / 4;
   if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, wrow / 4, a.N, wrow,
-                  static_cast<uint32_t>(gp_w_row_bytes(one_bit ? 2 : 0) / 4), static_cast<uint32_t>(kGpRows)) != TB_OK)
+                  static_cast<uint32_t>(gp_w_row_bytes(one_bit ? 2 : 0, false) / 4), static_cast<uint32_t>(kGpRows)) !=
+          TB_OK)
     return TB_ERR_CUDA;
   // y leaves through one TMA store per CTA where its rows are 16-byte aligned
   const int ysz = a.yt == TB_FP32 ? 4 : 2;
@@ -993,15 +994,15 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
 #define TB_GP_LAUNCH(BT, F)                                                                               \
   {                                                                                                       \
     if (a.yt == TB_FP32) {                                                                                \
-      auto k = gemm_pair_kernel<BT, float, F>;                                                            \
+      auto k = gemm_pair_kernel<BT, float, F, false>;                                                     \
       if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                  \
-      return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F)), a.st, tm_x, \
-                        tm_w, tm_y, gp, tma_y);                                                           \
+      return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, false)), a.st, \
+                        tm_x, tm_w, tm_y, gp, tma_y);                                                     \
     }                                                                                                     \
-    auto k = gemm_pair_kernel<BT, __nv_bfloat16, F>;                                                      \
+    auto k = gemm_pair_kernel<BT, __nv_bfloat16, F, false>;                                               \
     if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                    \
-    return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F)), a.st, tm_x,   \
-                      tm_w, tm_y, gp, tma_y);                                                             \
+    return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, false)), a.st,  \
+                      tm_x, tm_w, tm_y, gp, tma_y);                                                       \
   }
   if (bt == 128) {
     if (one_bit) TB_GP_LAUNCH(128, 2)
@@ -1040,43 +1041,47 @@ tb_status run_gemm_i8(const LinearArgs& a, const DevInfo* d) {
     return run_gemm_i8(c, d);
   }
   const bool one_bit = a.f == TB_FMT_1BIT;
-  int bm = 256, bn = 256;
-  gemm_tiles(a.M, a.N, d->sm_count, &bm, &bn);
-  CUtensorMap tm_x, tm_w;
-  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.x, a.K, a.M, a.K, kGi8BK, static_cast<uint32_t>(bm),
-                  CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
+  // the CTA-pair kernel of the fp16 GEMM in integer mode (kind::i8)
+  const int64_t pairs_n = (a.N + kGpPairRows - 1) / kGpPairRows;
+  const int bt = a.M <= 128 ? 128 : 256;
+  CUtensorMap tm_x, tm_w, tm_y;
+  if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.x, a.K, a.M, a.K, gp_atom_k(true),
+                  static_cast<uint32_t>(bt / 2), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
   const uint64_t wrow = one_bit ? a.K / 8 : a.K / 4;
   if (make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, wrow / 4, a.N, wrow,
-                  static_cast<uint32_t>(gi8_w_row_bytes(one_bit ? 2 : 0) / 4), static_cast<uint32_t>(bn)) != TB_OK)
+                  static_cast<uint32_t>(gp_w_row_bytes(one_bit ? 2 : 0, true) / 4), static_cast<uint32_t>(kGpRows)) !=
+      TB_OK)
     return TB_ERR_CUDA;
-  GemmI8Params gp;
+  int tma_y = 0;
+  tm_y = tm_x;
+  if (a.N % 4 == 0) {  // y rows 16-byte aligned (y itself is, by gemm_i8_ok)
+    if (make_map_2d(&tm_y, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, a.y, a.N, a.M, a.N * 4, static_cast<uint32_t>(kGpRows),
+                    static_cast<uint32_t>(bt)) != TB_OK)
+      return TB_ERR_CUDA;
+    tma_y = 1;
+  }
+  GemmParams gp;
   gp.M = static_cast<int>(a.M);
   gp.N = static_cast<int>(a.N);
   gp.K = static_cast<int>(a.K);
-  gp.y = static_cast<int32_t*>(a.y);
-  const dim3 grid(static_cast<unsigned>((a.N + bn - 1) / bn), static_cast<unsigned>((a.M + bm - 1) / bm));
-#define TB_GI8_F(BM, BN, F)                                                                                \
-  {                                                                                                        \
-    auto k = gemm_i8_kernel<BM, BN, F>;                                                                    \
-    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                     \
-    return launch_pdl(k, grid, dim3(kGemmThreads), static_cast<size_t>(gi8_smem_bytes(BM, BN, F)), a.st, tm_x, \
-                      tm_w, gp);                                                                           \
+  gp.y = a.y;
+  gp.scales = nullptr;
+  const dim3 grid(static_cast<unsigned>(2 * pairs_n), static_cast<unsigned>((a.M + bt - 1) / bt));
+#define TB_GI8_LAUNCH(BT, F)                                                                                  \
+  {                                                                                                           \
+    auto k = gemm_pair_kernel<BT, int32_t, F, true>;                                                          \
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                        \
+    return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, true)), a.st, tm_x, \
+                      tm_w, tm_y, gp, tma_y);                                                                 \
   }
-#define TB_GI8(BM, BN)                \
-  if (bm == BM && bn == BN) {         \
-    if (one_bit) TB_GI8_F(BM, BN, 2)  \
-    TB_GI8_F(BM, BN, 0)               \
+  if (bt == 128) {
+    if (one_bit) TB_GI8_LAUNCH(128, 2)
+    TB_GI8_LAUNCH(128, 0)
   }
-  TB_GI8(256, 256)
-  TB_GI8(256, 192)
-  TB_GI8(256, 128)
-  TB_GI8(128, 256)
-  TB_GI8(128, 192)
-  TB_GI8(128, 128)
-#undef TB_GI8
-#undef TB_GI8_F
-  return TB_ERR_SHAPE;
+  if (one_bit) TB_GI8_LAUNCH(256, 2)
+  TB_GI8_LAUNCH(256, 0)
+#undef TB_GI8_LAUNCH
 }
 
 bool known_format(int f) { return f == TB_FMT_2BIT || f == TB_FMT_BASE3 || f == TB_FMT_1BIT; }
