@@ -480,7 +480,8 @@ def run_prefill(args, dev, stream, tb, inputs, world=1, integer=False):
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": round(peak, 1),
                          "unit": "TFLOP/s" if not integer else "TOP/s", "frac": round(tflops / peak, 4),
                          "peak_source": kind,
-                         "dtype": "s8 x u8 -> s32 (kind::i8)" if integer else "fp16 x fp16 -> fp32 (kind::f16)"},
+                         "dtype": "s8 x s8 -> s32 (kind::i8)" if integer else "fp16 x fp16 -> fp32 (kind::f16)",
+                         "kernel": "gemm_pair_kernel (CTA pairs, cta_group::2, A = unpacked weights in TMEM)"},
             "clocks": clocks,
             "kernel_path": tb.tb_ternary_linear_path(xt, "2bit", m, n, k, not integer, True)}
 

@@ -107,12 +107,13 @@ typedef int tb_path;
                             of 4 tokens; 1-bit: M = 1).  One token (2-bit,
                             1-bit): one launch that rotates x itself for
                             K <= 8192                                          */
-#define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel (fp16 x' times exact fp16
-                            s*t in shared memory, fp32 accumulators in TMEM;
-                            integer mode: kind::i8, int8 x times the biased
-                            codes, exact int32 accumulators, from 16 tokens,
-                            any K % 128, base-3 only with a workspace to
-                            re-encode into);
+#define TB_PATH_GEMM 2   /* tcgen05 tensor-core kernel on CTA pairs (weights
+                            unpacked into TMEM as the A operand: exact fp16
+                            s*t against fp16 x', fp32 accumulators; integer
+                            mode: kind::i8, the ternary codes as signed bytes
+                            against int8 x, exact int32 accumulators, from 16
+                            tokens, any K % 128, base-3 only with a workspace
+                            to re-encode into);
                             base-3 from 8 tokens, re-encoded to 2-bit slots in
                             the workspace first; 1-bit from 2 tokens.  Chosen
                             by TB_PATH_AUTO past 16 tokens, or from 8 base-3

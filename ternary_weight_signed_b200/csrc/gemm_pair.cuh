@@ -42,12 +42,69 @@
 // word and still reaches the final cluster barrier, so no CTA leaves while its
 // peer may touch its memory, and TMEM is always freed.
 #pragma once
-#include "gemm_i8.cuh"
-#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
+#include "hadamard.cuh"
+#include "tcgen05.cuh"
 
 namespace tb {
+
+// ---------------------------------------------------------------------------
+// Activation prep of the fp16 GEMM: rotation (when signs is non-null) and an
+// fp16 store in the paired order inside every 16-element chunk (k = 0, 8, 1,
+// 9, ..., 7, 15), the order the unpack writes the weights in.  grid (M,
+// K/1024), 128 threads.
+template <typename TIn>
+__global__ void __launch_bounds__(kHThreads) prep_gemm_kernel(const TIn* __restrict__ x,
+                                                              const int8_t* __restrict__ signs,
+                                                              __half* __restrict__ out, int64_t K) {
+  __shared__ float sm[kHB];
+  pdl_launch_dependents();
+  const int64_t row = blockIdx.x;
+  const int blk = blockIdx.y;
+  float v[8];
+  load_rotated8<TIn>(x, signs, row, blk, K, v, sm);
+  // thread pair (2c, 2c+1) holds the 16-element chunk c; exchange halves
+  const bool upper = (threadIdx.x & 1) != 0;
+  float u[4], p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) u[i] = upper ? v[i] : v[4 + i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = __shfl_xor_sync(0xffffffffu, u[i], 1);
+  float o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = upper ? p[i] : v[i];
+    o[2 * i + 1] = upper ? v[4 + i] : p[i];
+  }
+  store8<__half>(out + row * K + static_cast<int64_t>(blk) * kHB + 8 * threadIdx.x, o);
+}
+
+struct GemmParams {
+  int M, N, K;
+  void* y;
+  const uint16_t* scales;  // [N, K/128] fp16 bits
+};
+
+// 16 codes of a 2-bit word (code u in bits 2u) as 16 bytes c_u = t_u + 1 in
+// natural order: the masks m_j = (w >> 2j) & 0x03030303 hold c_{4b+j} in byte
+// b; a 4 x 4 byte transpose (eight byte permutes) gives (c_{4b}, .., c_{4b+3}).
+__device__ __forceinline__ uint4 gi8_codes16(uint32_t w) {
+  const uint32_t m0 = w & 0x03030303u, m1 = (w >> 2) & 0x03030303u, m2 = (w >> 4) & 0x03030303u,
+                 m3 = (w >> 6) & 0x03030303u;
+  const uint32_t a_lo = __byte_perm(m0, m1, 0x5140), a_hi = __byte_perm(m0, m1, 0x7362);  // c0 c1 c4 c5 | c8 ..
+  const uint32_t b_lo = __byte_perm(m2, m3, 0x5140), b_hi = __byte_perm(m2, m3, 0x7362);  // c2 c3 c6 c7 | c10 ..
+  return make_uint4(__byte_perm(a_lo, b_lo, 0x5410), __byte_perm(a_lo, b_lo, 0x7632), __byte_perm(a_hi, b_hi, 0x5410),
+                    __byte_perm(a_hi, b_hi, 0x7632));
+}
+
+// Four 1-bit codes (bits 4r .. 4r + 3 of w) as four bytes b in {0, 1}: the
+// product with 0x00204081 places bit i of the nibble at bit 8 i (the four
+// shifted copies occupy disjoint bit ranges, so nothing carries).
+__device__ __forceinline__ uint32_t gi8_bits4(uint32_t w, int r) {
+  return (((w >> (4 * r)) & 0xFu) * 0x00204081u) & 0x01010101u;
+}
+
 
 constexpr int kGpSets = 4;  // unpack warp sets (stage kb goes to set kb % 4)
 constexpr int kGpThreads = 32 * (2 + 4 * kGpSets);

@@ -34,7 +34,7 @@
 // them in a fixed order, so the result does not depend on timing.  With more
 // rows than 148 * 128, a CTA runs T = 2 or more tiles in turn.
 #pragma once
-#include "gemm_tc.cuh"
+#include "tcgen05.cuh"
 #include "hadamard.cuh"
 #include "tb_device.cuh"
 

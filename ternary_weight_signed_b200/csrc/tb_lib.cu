@@ -14,9 +14,7 @@
 #include "ternary_b200.h"
 #include "tb_device.cuh"
 
-#include "gemm_tc.cuh"
 #include "gemm_pair.cuh"
-#include "gemm_i8.cuh"
 #include "gemv.cuh"
 #include "gemv_m1.cuh"
 #include "prepare.cuh"
@@ -517,7 +515,7 @@ bool gemm_ok(const LinearArgs& a) {
   // decode comes first where its row limit allows)
   if (a.f == TB_FMT_BASE3 && a.M < kB3TranscodeMinM) return false;
   return is_float_dtype(a.xt) && a.K % 1024 == 0 && fast_aligned(a) &&
-         (a.M + kGemmUM - 1) / kGemmUM <= 65535 && a.N < (int64_t(1) << 30);
+         (a.M + 127) / 128 <= 65535 && a.N < (int64_t(1) << 30);
 }
 
 bool gemm_i8_ok(const LinearArgs& a);
@@ -921,34 +919,6 @@ tb_status run_gemm(const LinearArgs& a, const DevInfo* d) {
   return run_gemm_2bit(c, d);
 }
 
-// Tiles of the tensor-core GEMMs.  Token tile: 128 when it pads fewer token
-// rows than 256 (up to 128 tokens, and e.g. 300 tokens: 384 against 512 rows),
-// else 256, whose two MMAs share each unpacked weight tile.  Weight-tile
-// width: wave fill of the SMs times the tile's own efficiency.  Narrower tiles
-// reuse each activation stage for fewer weight rows and leave unpack warps
-// idle; on B200 the 192-wide tile ran the prefill shape (2048 x 17408 x 5120)
-// at 0.90 of the 256-wide tile's per-tile rate, which its better wave fill
-// (4.92 against 3.68 waves) does not make up.
-void gemm_tiles(int64_t M, int64_t N, int sm_count, int* bm_out, int* bn_out) {
-  const int bm = ((M + 127) / 128) * 128 < ((M + 255) / 256) * 256 ? 128 : 256;
-  const int64_t mt = (M + bm - 1) / bm;
-  int bn = 256;
-  double best = -1.0;
-  const int cands[3] = {256, 192, 128};
-  const double eff[3] = {1.0, 0.9, 0.8};
-  for (int i = 0; i < 3; ++i) {
-    const double tiles = static_cast<double>(((N + cands[i] - 1) / cands[i]) * mt);
-    const double waves = tiles / sm_count;
-    const double score = eff[i] * waves / std::ceil(waves);
-    if (score > best + 1e-9) {
-      best = score;
-      bn = cands[i];
-    }
-  }
-  *bm_out = bm;
-  *bn_out = bn;
-}
-
 // 2-bit slots or 1-bit codes (base-3 arrives re-encoded to 2-bit slots).
 tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
   const bool one_bit = a.f == TB_FMT_1BIT;
@@ -1019,7 +989,7 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
 constexpr int kGi8MinM = 16;
 
 bool gemm_i8_ok(const LinearArgs& a) {
-  if (a.xt != TB_INT8 || a.M < kGi8MinM || a.K % kGi8BK != 0 || (a.M + kGemmUM - 1) / kGemmUM > 65535 ||
+  if (a.xt != TB_INT8 || a.M < kGi8MinM || a.K % 128 != 0 || (a.M + 127) / 128 > 65535 ||
       a.N >= (int64_t(1) << 30))
     return false;
   if (!(aligned(a.x, 16) && aligned(a.packed, 16) && aligned(a.y, 16))) return false;
