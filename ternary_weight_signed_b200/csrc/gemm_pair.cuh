@@ -9,31 +9,41 @@
 // come by TMA into shared memory as operand B.  So shared memory carries only
 // the x' tiles and the packed codes; the fp16 weights never touch it.
 //
-// One pair tile is 256 weight rows x BT tokens (BT = 128, 192 or 256, chosen
-// per shape for whole waves).  CTA r of the cluster owns weight rows 128 r .. 128 r + 127 (its
-// TMEM lanes) and loads tokens BT/2 r .. BT/2 r + BT/2 - 1 of the x' tile; one
-// M = 256 MMA issued by CTA 0 multiplies both CTAs' A (TMEM) by the B halves
-// of both CTAs, and each CTA's TMEM receives D for its own 128 weight rows and
-// all BT tokens.  Per K step of 16 a CTA's shared memory is read for BT/2
+// One pair tile is 256 weight rows x BT tokens (BT = 256, or 128 up to 128
+// tokens).  CTA r of the cluster owns weight rows 128 r .. 128 r + 127 of the
+// tile (its TMEM lanes) and loads tokens BT/2 r .. BT/2 r + BT/2 - 1 of the x'
+// tile; one M = 256 MMA issued by CTA 0 multiplies both CTAs' A (TMEM) by the
+// B halves of both CTAs, and each CTA's TMEM receives D for its own 128 weight
+// rows and all BT tokens.  Per K step a CTA's shared memory is read for BT/2
 // tokens only, half of what a one-CTA MMA of the same width reads.
+//
+// The kernel is persistent: one cluster per SM pair at most, each walking its
+// tiles with one continuous stage sequence, so the copies and the unpack of a
+// tile's first stages overlap the previous tile's last MMAs, and its MMAs wait
+// only until every warp has read the previous tile's D into registers.
 //
 // Warp roles in each CTA:
 //   warp 0     : TMA producer (x' half tile with 128B swizzle; packed codes);
 //   warp 1     : TMEM allocation for the pair; in CTA 0, the thread issuing
 //                the MMAs;
 //   warps 2-17 : unpack, four sets of four warps: warp w takes TMEM lanes
-//                32 (w % 4) .. + 31 and the stages kb = j, j + 4, ... of its
-//                set j = (w - 2) / 4, so each warp has four stages of MMA time
-//                for the fixed cost of one (barrier waits, the hand-off);
-//                then the epilogue (tcgen05.ld of D, convert, store y with
-//                the weight rows along the warp's lanes).
-// Hand-offs per stage s:
-//   full[s]  (each CTA): the CTA's x' half and codes landed (TMA);
-//   ready[s] (CTA 0)   : the 8 unpack warps of both CTAs wrote their A
-//                        slices and saw their x' half land (the other CTA's
-//                        warps arrive through the cluster's shared window);
-//   empty[s] (each CTA): the stage's MMAs are done (commit multicast to both
-//                        CTAs) - its x' half, codes and TMEM A slice are free.
+//                32 (w % 4) .. + 31 and the stages g = j, j + 4, ... of its
+//                set j = (w - 2) / 4 (A slot j), so each warp has four stages
+//                of MMA time for the fixed cost of one (barrier waits, the
+//                hand-off).  Right after its first stage of a tile, a warp
+//                reads its quarter of the previous tile's D (its 32 lanes, BT/4
+//                columns), releases D and stores y, the weight rows along the
+//                warp's lanes.
+// Hand-offs:
+//   full[s]  (each CTA, shared-memory slot): x' half and codes landed (TMA);
+//   sfree[s] (each CTA): the slot's MMAs are done (commit multicast to both
+//            CTAs) and the unpack warps hold its codes in registers;
+//   ready[a] (CTA 0, TMEM A slot): the 8 warps of the set, 4 per CTA, wrote the
+//            slot and saw their x' half land (the other CTA's warps arrive
+//            through the cluster's shared window);
+//   afree[a] (each CTA): the MMAs reading the A slot are done (multicast);
+//   accum    (each CTA): the tile's MMAs are done; dfree (CTA 0): all 32
+//            unpack warps read D out.
 // The code order inside a 16-code chunk is the one the prep kernel writes x'
 // in (k = 0, 8, 1, 9, ..., 7, 15): the TMEM column j of a chunk holds the fp16
 // pair (w_j, w_{j+8}).
@@ -213,55 +223,20 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       "h"(static_cast<uint16_t>(3))
       : "memory");
 }
-template <typename TOut>
-__device__ __forceinline__ void store_out(TOut* p, uint32_t v);
-template <>
-__device__ __forceinline__ void store_out<float>(float* p, uint32_t v) {
-  *p = __uint_as_float(v);
-}
-template <>
-__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, uint32_t v) {
-  *p = __float2bfloat16_rn(__uint_as_float(v));
-}
-template <>
-__device__ __forceinline__ void store_out<int32_t>(int32_t* p, uint32_t v) {
-  *p = static_cast<int32_t>(v);
-}
-
-// 2-D tiled store of one box from shared memory (bulk group of this thread).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
-               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
-               : "memory");
-}
-// Named barrier `id` over `count` threads that also ANDs a predicate.
-__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void bulk_commit_and_wait_read() {
-  asm volatile(
-      "cp.async.bulk.commit_group;\n\t"
-      "cp.async.bulk.wait_group.read 0;" ::
-          : "memory");
-}
+// Tiles of one launch: tiles_n weight-row pairs x tiles_m token tiles, taken
+// in order t = tn + tiles_n * tm by the clusters in turn (cluster c: t = c,
+// c + C, ...), so that the clusters running at one time share token tiles.
+struct GemmPairTiles {
+  int tiles_n, tiles_m;
+};
 
 // kFmt: 0 = 2-bit slots, 2 = 1-bit g128.  kInt: integer mode (int8 x, no
 // rotation, no scales, exact int32 y; A = t as signed bytes), else fp16 x' and
-// A = fp16(s t).  tma_y: y goes out through shared memory and one TMA store
-// per CTA (rows 16-byte aligned), else by plain stores.
+// A = fp16(s t).
 template <int BT, typename TOut, int kFmt, bool kInt>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                     const __grid_constant__ CUtensorMap tm_y, const GemmParams p, const int tma_y) {
+                     const GemmParams p, const GemmPairTiles tl) {
   static_assert(kFmt == 0 || kFmt == 2, "2-bit or 1-bit codes");
   static_assert(BT % 64 == 0 && BT >= 128 && BT <= kGpDCols, "token tile");
   constexpr int kBK = gp_bk(kInt), kAtomK = gp_atom_k(kInt), kWr = gp_w_row_bytes(kFmt, kInt);
@@ -269,23 +244,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
   constexpr int kStage = gp_stage_bytes(BT, kFmt, kInt), S = gp_stages(BT, kFmt, kInt), SA = kGpASlots;
   static_assert(kAtom % 1024 == 0 && kStage % 1024 == 0, "128B-swizzle atoms stay 1024-byte aligned");
   static_assert(S >= SA, "the copies run at least as far ahead as the unpack");
-  static_assert(BT * kGpRows * static_cast<int>(sizeof(TOut)) <= S * kStage, "the y tile fits the stage ring");
   constexpr uint32_t kIdesc = gp_idesc(BT, kInt);
+  constexpr int kCols = BT / kGpSets;  // D columns (tokens) one unpack warp reads out
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kStage);  // copies landed
-  uint64_t* sfree = full + S;   // stage slot read: by the MMAs (x') and the unpack warps (codes)
-  uint64_t* ready = sfree + S;  // (CTA 0) A slot written and x' landed, in both CTAs
-  uint64_t* afree = ready + SA; // the MMAs reading an A slot are done
-  uint64_t* accum = afree + SA;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* sfree = full + S;    // stage slot read: by the MMAs (x) and the unpack warps (codes)
+  uint64_t* ready = sfree + S;   // (CTA 0) A slot written and x landed, in both CTAs
+  uint64_t* afree = ready + SA;  // the MMAs reading an A slot are done
+  uint64_t* accum = afree + SA;  // a tile's MMAs are done (D complete)
+  uint64_t* dfree = accum + 1;   // (CTA 0) D read out by every unpack warp of both CTAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dfree + 1);
 
   const uint32_t rank = cluster_rank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = static_cast<int>(blockIdx.x >> 1) * kGpPairRows + static_cast<int>(rank) * kGpRows;
-  const int m0 = blockIdx.y * BT;
+  const int cluster = static_cast<int>(blockIdx.x >> 1), nclusters = static_cast<int>(gridDim.x >> 1);
+  const int ntiles = tl.tiles_n * tl.tiles_m;
+  const int mine = (ntiles - cluster + nclusters - 1) / nclusters;  // tiles of this cluster
   // integer mode: K a multiple of 128; a last half stage reads zeros past K
   const int nk = (p.K + kBK - 1) / kBK;
+  auto tile_n0 = [&](int i) {  // this CTA's first weight row in its i-th tile
+    return ((cluster + i * nclusters) % tl.tiles_n) * kGpPairRows + static_cast<int>(rank) * kGpRows;
+  };
+  auto tile_m0 = [&](int i) { return ((cluster + i * nclusters) / tl.tiles_n) * BT; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -297,6 +278,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
       mbar_init(&afree[a], 1);
     }
     mbar_init(accum, 1);
+    mbar_init(dfree, 2 * 4 * kGpSets);  // every unpack warp of both CTAs
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -314,53 +296,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&tm_x);
       prefetch_tensormap(&tm_w);
-      pdl_wait();  // x' comes from the prep kernel
+      pdl_wait();  // x comes from the previous kernel (the prep kernel, in float mode)
       const bool stall = test_stall_copies();  // failure-detection test: no copies
-      int issued = 0;
-      for (int kb = 0; kb < nk && !stall; ++kb) {
-        const int s = kb % S;
-        if (kb >= S && !mbar_wait(&sfree[s], ((kb / S) & 1) ^ 1, FAULT_WAIT_EMPTY)) break;
-        uint8_t* st = smem + s * kStage;
-        mbar_arrive_expect_tx(&full[s], kX + kW);
-        const int my = m0 + static_cast<int>(rank) * (BT / 2);
-        tma_load_2d(st, &tm_x, kb * kBK, my, &full[s]);
-        tma_load_2d(st + kAtom, &tm_x, kb * kBK + kAtomK, my, &full[s]);
-        // x in 32-bit words: the codes of a stage are kWr bytes of each row
-        tma_load_2d(st + kX, &tm_w, kb * (kWr / 4), n0, &full[s]);
-        issued = kb + 1;
+      int g = 0;     // stage counter over all tiles of this cluster
+      bool ok = !stall;
+      for (int i = 0; i < mine && ok; ++i) {
+        const int n0 = tile_n0(i), my = tile_m0(i) + static_cast<int>(rank) * (BT / 2);
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = g % S;
+          if (g >= S && !mbar_wait(&sfree[s], ((g / S) & 1) ^ 1, FAULT_WAIT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStage;
+          mbar_arrive_expect_tx(&full[s], kX + kW);
+          tma_load_2d(st, &tm_x, kb * kBK, my, &full[s]);
+          tma_load_2d(st + kAtom, &tm_x, kb * kBK + kAtomK, my, &full[s]);
+          // x in 32-bit words: the codes of a stage are kWr bytes of each row
+          tma_load_2d(st + kX, &tm_w, kb * (kWr / 4), n0, &full[s]);
+        }
       }
       // the last copies issued land before the CTA may leave
-      for (int kb = issued > S ? issued - S : 0; kb < issued; ++kb)
-        if (!mbar_wait(&full[kb % S], (kb / S) & 1, FAULT_WAIT_FULL)) break;
+      for (int h = g > S ? g - S : 0; h < g; ++h)
+        if (!mbar_wait(&full[h % S], (h / S) & 1, FAULT_WAIT_FULL)) break;
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA (CTA 0)
     if (rank == 0 && lane == 0) {
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S, a = kb % SA;
-        if (!mbar_wait(&ready[a], (kb / SA) & 1, FAULT_WAIT_FULL)) break;
-        tc_fence_after();
-        const uint32_t b = smem_u32(smem + s * kStage);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < mine && ok; ++i) {
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = g % S, a = g % SA;
+          if (!mbar_wait(&ready[a], (g / SA) & 1, FAULT_WAIT_FULL)) {
+            ok = false;
+            break;
+          }
+          // the first MMA of a tile overwrites D: every warp has read out the last tile's
+          if (kb == 0 && i > 0 && !mbar_wait(dfree, (i - 1) & 1, FAULT_WAIT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b = smem_u32(smem + s * kStage);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_pair_ts<kInt>(tmem_d, tmem_a + static_cast<uint32_t>(a * kGpACols + 8 * kk),
-                           umma_desc_sw128(b + (kk >> 2) * kAtom + 32 * (kk & 3)), kIdesc,
-                           (kb | kk) != 0 ? 1u : 0u);
-        umma_commit_pair(&sfree[s]);
-        umma_commit_pair(&afree[a]);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_pair_ts<kInt>(tmem_d, tmem_a + static_cast<uint32_t>(a * kGpACols + 8 * kk),
+                               umma_desc_sw128(b + (kk >> 2) * kAtom + 32 * (kk & 3)), kIdesc,
+                               (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(&sfree[s]);
+          umma_commit_pair(&afree[a]);
+        }
+        umma_commit_pair(accum);
       }
-      umma_commit_pair(accum);
+      if (!ok) umma_commit_pair(accum);  // whoever waits for the tile stops waiting
     }
   } else {
-    // ---------------------------------------------------------------- unpack
+    // ---------------------------------------------------------------- unpack + read-out
     const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int set = (warp - 2) >> 2;   // stages set, set + 4, ... (A slot set)
+    const int set = (warp - 2) >> 2;   // stages g = set, set + 4, ... (A slot set)
     const int r = 32 * q + lane;       // weight row of this CTA = TMEM lane
-    const int n = n0 + r;
-    const bool row_ok = n < p.N;
     const int G = p.K / 128;
-    const bool scaled = !kInt && row_ok;  // integer mode has no scales
-    const uint16_t* srow = kInt ? nullptr : p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
     const __half2 k1024 = __float2half2_rn(1024.f);
     const __half2 k1 = __float2half2_rn(1.f);
     const __half2 kinv256 = __float2half2_rn(1.f / 256.f);
@@ -368,47 +364,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     const uint32_t ta = tmem_a + lane_addr + static_cast<uint32_t>(set * kGpACols);
     const uint32_t ready0 = cluster_map(smem_u32(&ready[set]), 0);  // CTA 0's ready barrier of this set
-    uint16_t s_bits = (scaled && set < nk) ? srow[set] : uint16_t(0);  // fp16: stage kb is scale group kb
-    for (int kb = set; kb < nk; kb += kGpSets) {
-      const int s = kb % S;
-      const int kn = kb + kGpSets;  // this warp's next stage: its scale is loaded a stage early
-      const uint16_t s_nb = (scaled && kn < nk) ? srow[kn] : uint16_t(0);
+    const uint32_t dfree0 = cluster_map(smem_u32(dfree), 0);
+    bool ok = true;
+    int done = 0;  // tiles whose D this warp has read out and stored
+    // D of tile `done` -> registers (then D is released) -> y
+    auto read_out = [&]() {
+      const bool got = __all_sync(0xffffffffu, mbar_wait(accum, done & 1, FAULT_WAIT_EPILOGUE));
+      if (!got) {
+        ok = false;
+        return;
+      }
+      tc_fence_after();
+      // 16-bit outputs are converted as they come (pairs of tokens in one
+      // register), so the warp holds half as many registers until D is free
+      constexpr bool kPack = sizeof(TOut) == 2;
+      uint32_t h[kPack ? kCols / 2 : kCols];
+#pragma unroll
+      for (int c = 0; c < kCols; c += 32) {
+        uint32_t v[32];
+        tmem_ld_cols<32>(tmem_d + lane_addr + static_cast<uint32_t>(set * kCols + c), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          if constexpr (kPack) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            h[(c + j) / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+          } else {
+            h[c + j] = v[j];
+            h[c + j + 1] = v[j + 1];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(dfree0);
+      const int n = tile_n0(done) + r, mb = tile_m0(done) + set * kCols;
+      if (n < p.N) {
+        TOut* y = reinterpret_cast<TOut*>(p.y) + n;
+#pragma unroll
+        for (int j = 0; j < kCols; ++j) {
+          if (mb + j >= p.M) break;
+          TOut* dst = y + static_cast<int64_t>(mb + j) * p.N;
+          if constexpr (kPack)
+            *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(h[j / 2] >> (16 * (j & 1)));
+          else
+            *reinterpret_cast<uint32_t*>(dst) = h[j];
+        }
+      }
+      ++done;
+    };
+    const int total = mine * nk;
+    for (int g = set; g < total && ok; g += kGpSets) {
+      const int i = g / nk, kb = g - i * nk, s = g % S;
+      // read out every tile before the last one first (a set may have no stage in a tile)
+      while (ok && done < i - 1) read_out();
+      if (!ok) break;
+      const int n = tile_n0(i) + r;
+      const bool row_ok = n < p.N;
+      // this stage's scale (fp16 mode: stage kb is scale group kb)
+      const uint16_t s_bits = (!kInt && row_ok) ? p.scales[static_cast<int64_t>(n) * G + kb] : uint16_t(0);
       // every lane waits (each reads the stage); the warp leaves together
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (kb / S) & 1, FAULT_WAIT_FULL))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1, FAULT_WAIT_FULL))) {
+        ok = false;
+        break;
+      }
       const uint8_t* wrow = smem + s * kStage + kX + r * kWr;
       uint4 wv[kWr / 16];
 #pragma unroll
-      for (int i = 0; i < kWr / 16; ++i) wv[i] = *reinterpret_cast<const uint4*>(wrow + 16 * i);
+      for (int u = 0; u < kWr / 16; ++u) wv[u] = *reinterpret_cast<const uint4*>(wrow + 16 * u);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sfree[s]);  // the codes are in registers
-      // the MMAs of stage kb - 4 are done with this A slot
-      if (kb >= SA && !__all_sync(0xffffffffu, mbar_wait(&afree[set], ((kb / SA) & 1) ^ 1, FAULT_WAIT_MMA)))
+      // the MMAs of stage g - 4 are done with this A slot
+      if (g >= SA && !__all_sync(0xffffffffu, mbar_wait(&afree[set], ((g / SA) & 1) ^ 1, FAULT_WAIT_MMA))) {
+        ok = false;
         break;
+      }
       tc_fence_after();
       const __half sc = __ushort_as_half(s_bits);
       const __half2 s2 = __halves2half2(sc, sc);
       const __half2 ns2 = __hneg2(s2);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {  // codes 64 half .. 64 half + 63 -> 32 TMEM columns
+      for (int half = 0; half < 2; ++half) {  // codes of half the stage -> 32 TMEM columns
         uint32_t o[32];
         if constexpr (kInt && kFmt == 0) {
           // codes 128 half .. + 127: packed words 8 half .. + 7, each as 16
           // bytes c = t + 1 in natural order, then t = c - 1 bytewise:
           // (c + 0x7F) ^ 0x80 never carries out of a byte (c <= 2)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint4 c4 = gi8_codes16((&wv[0].x)[8 * half + i]);
+          for (int u = 0; u < 8; ++u) {
+            const uint4 c4 = gi8_codes16((&wv[0].x)[8 * half + u]);
 #pragma unroll
-            for (int b = 0; b < 4; ++b) o[4 * i + b] = ((&c4.x)[b] + 0x7F7F7F7Fu) ^ 0x80808080u;
+            for (int b = 0; b < 4; ++b) o[4 * u + b] = ((&c4.x)[b] + 0x7F7F7F7Fu) ^ 0x80808080u;
           }
         } else if constexpr (kInt) {
           // 1-bit: codes 128 half .. + 127 are words 4 half .. + 3, 32 codes a
           // word; t = 2 b - 1 bytewise as (2 b + 0x7F) ^ 0x80
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t w = (&wv[0].x)[4 * half + i];
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t w = (&wv[0].x)[4 * half + u];
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) o[8 * i + rr] = ((gi8_bits4(w, rr) << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
+            for (int rr = 0; rr < 8; ++rr) o[8 * u + rr] = ((gi8_bits4(w, rr) << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
           }
         } else if constexpr (kFmt == 2) {
           // chunk c of the 128 codes (16 codes) is half c & 1 of word c >> 1.
@@ -447,48 +502,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGpThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(ready0);
-      s_bits = s_nb;
+      // right after this warp's first stage of a tile, the previous tile's D
+      while (ok && done < i) read_out();
     }
-    // ---------------------------------------------------------------- epilogue
-    constexpr int kEpiThreads = 4 * kGpSets * 32;
-    // one decision for all epilogue warps (they meet at a named barrier below)
-    if (bar_and(1, kEpiThreads, mbar_wait(accum, 0, FAULT_WAIT_EPILOGUE))) {
-      tc_fence_after();
-      constexpr int kCols = BT / kGpSets;  // tokens of this warp: set * kCols .. + kCols - 1
-      if (tma_y) {
-        // y tile [BT tokens][128 rows] in the (now idle) stage ring, then one
-        // TMA store, which also drops what lies beyond M or N
-        TOut* ty = reinterpret_cast<TOut*>(smem);
-#pragma unroll 1
-        for (int c0 = set * kCols; c0 < (set + 1) * kCols; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld_cols<16>(tmem_d + lane_addr + static_cast<uint32_t>(c0), v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) store_out<TOut>(ty + (c0 + j) * kGpRows + r, v[j]);
-        }
-        fence_proxy_async_shared();  // generic-proxy stores -> visible to the TMA store
-        asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-        if (warp == 2 && lane == 0 && n0 < p.N) {  // a CTA past the last row has nothing to store
-          tma_store_2d(&tm_y, ty, n0, m0);
-          bulk_commit_and_wait_read();
-        }
-      } else {
-        TOut* y = reinterpret_cast<TOut*>(p.y) + n;
-#pragma unroll 1
-        for (int c0 = set * kCols; c0 < (set + 1) * kCols; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld_cols<16>(tmem_d + lane_addr + static_cast<uint32_t>(c0), v);
-          tmem_ld_wait();
-          const int mb = m0 + c0;
-          if (row_ok) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (mb + j < p.M) store_out<TOut>(y + static_cast<int64_t>(mb + j) * p.N, v[j]);
-          }
-        }
-      }
-    }
+    while (ok && done < mine) read_out();
   }
   __syncwarp();
   tc_fence_before();

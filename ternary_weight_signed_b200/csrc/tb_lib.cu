@@ -515,7 +515,8 @@ bool gemm_ok(const LinearArgs& a) {
   // decode comes first where its row limit allows)
   if (a.f == TB_FMT_BASE3 && a.M < kB3TranscodeMinM) return false;
   return is_float_dtype(a.xt) && a.K % 1024 == 0 && fast_aligned(a) &&
-         (a.M + 127) / 128 <= 65535 && a.N < (int64_t(1) << 30);
+         (a.M + 127) / 128 <= 65535 && a.N < (int64_t(1) << 30) &&
+         ((a.N + 255) / 256) * ((a.M + 127) / 128) < (int64_t(1) << 31);  // tile indices fit an int
 }
 
 bool gemm_i8_ok(const LinearArgs& a);
@@ -944,35 +945,30 @@ tb_status run_gemm_2bit(const LinearArgs& a, const DevInfo* d) {
                   static_cast<uint32_t>(gp_w_row_bytes(one_bit ? 2 : 0, false) / 4), static_cast<uint32_t>(kGpRows)) !=
           TB_OK)
     return TB_ERR_CUDA;
-  // y leaves through one TMA store per CTA where its rows are 16-byte aligned
-  const int ysz = a.yt == TB_FP32 ? 4 : 2;
-  CUtensorMap tm_y = tm_x;
-  int tma_y = 0;
-  if (aligned(a.y, 16) && (a.N * ysz) % 16 == 0) {
-    if (make_map_2d(&tm_y, a.yt == TB_FP32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ysz,
-                    a.y, a.N, a.M, a.N * ysz, static_cast<uint32_t>(kGpRows), static_cast<uint32_t>(bt)) != TB_OK)
-      return TB_ERR_CUDA;
-    tma_y = 1;
-  }
   GemmParams gp;
   gp.M = static_cast<int>(a.M);
   gp.N = static_cast<int>(a.N);
   gp.K = static_cast<int>(a.K);
   gp.y = a.y;
   gp.scales = a.scales;
-  const dim3 grid(static_cast<unsigned>(2 * pairs_n), static_cast<unsigned>((a.M + bt - 1) / bt));
-#define TB_GP_LAUNCH(BT, F)                                                                               \
-  {                                                                                                       \
-    if (a.yt == TB_FP32) {                                                                                \
-      auto k = gemm_pair_kernel<BT, float, F, false>;                                                     \
-      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                  \
-      return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, false)), a.st, \
-                        tm_x, tm_w, tm_y, gp, tma_y);                                                     \
-    }                                                                                                     \
-    auto k = gemm_pair_kernel<BT, __nv_bfloat16, F, false>;                                               \
-    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                    \
-    return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, false)), a.st,  \
-                      tm_x, tm_w, tm_y, gp, tma_y);                                                       \
+  GemmPairTiles tl;
+  tl.tiles_n = static_cast<int>(pairs_n);
+  tl.tiles_m = static_cast<int>((a.M + bt - 1) / bt);
+  // persistent: one cluster per SM pair at most, each walking its tiles
+  const int64_t ntiles = pairs_n * tl.tiles_m;
+  const dim3 grid(static_cast<unsigned>(2 * std::min<int64_t>(ntiles, std::max(1, d->sm_count / 2))));
+#define TB_GP_LAUNCH(BT, F)                                                                                   \
+  {                                                                                                           \
+    if (a.yt == TB_FP32) {                                                                                    \
+      auto k = gemm_pair_kernel<BT, float, F, false>;                                                         \
+      if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                      \
+      return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, false)), a.st,    \
+                        tm_x, tm_w, gp, tl);                                                                  \
+    }                                                                                                         \
+    auto k = gemm_pair_kernel<BT, __nv_bfloat16, F, false>;                                                   \
+    if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                        \
+    return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, false)), a.st, tm_x, \
+                      tm_w, gp, tl);                                                                          \
   }
   if (bt == 128) {
     if (one_bit) TB_GP_LAUNCH(128, 2)
@@ -990,7 +986,7 @@ constexpr int kGi8MinM = 16;
 
 bool gemm_i8_ok(const LinearArgs& a) {
   if (a.xt != TB_INT8 || a.M < kGi8MinM || a.K % 128 != 0 || (a.M + 127) / 128 > 65535 ||
-      a.N >= (int64_t(1) << 30))
+      a.N >= (int64_t(1) << 30) || ((a.N + 255) / 256) * ((a.M + 127) / 128) >= (int64_t(1) << 31))
     return false;
   if (!(aligned(a.x, 16) && aligned(a.packed, 16) && aligned(a.y, 16))) return false;
   // base-3: re-encoded to 2-bit slots first, in a workspace the caller passed
@@ -1014,7 +1010,7 @@ tb_status run_gemm_i8(const LinearArgs& a, const DevInfo* d) {
   // the CTA-pair kernel of the fp16 GEMM in integer mode (kind::i8)
   const int64_t pairs_n = (a.N + kGpPairRows - 1) / kGpPairRows;
   const int bt = a.M <= 128 ? 128 : 256;
-  CUtensorMap tm_x, tm_w, tm_y;
+  CUtensorMap tm_x, tm_w;
   if (make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.x, a.K, a.M, a.K, gp_atom_k(true),
                   static_cast<uint32_t>(bt / 2), CU_TENSOR_MAP_SWIZZLE_128B) != TB_OK)
     return TB_ERR_CUDA;
@@ -1023,27 +1019,23 @@ tb_status run_gemm_i8(const LinearArgs& a, const DevInfo* d) {
                   static_cast<uint32_t>(gp_w_row_bytes(one_bit ? 2 : 0, true) / 4), static_cast<uint32_t>(kGpRows)) !=
       TB_OK)
     return TB_ERR_CUDA;
-  int tma_y = 0;
-  tm_y = tm_x;
-  if (a.N % 4 == 0) {  // y rows 16-byte aligned (y itself is, by gemm_i8_ok)
-    if (make_map_2d(&tm_y, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, a.y, a.N, a.M, a.N * 4, static_cast<uint32_t>(kGpRows),
-                    static_cast<uint32_t>(bt)) != TB_OK)
-      return TB_ERR_CUDA;
-    tma_y = 1;
-  }
   GemmParams gp;
   gp.M = static_cast<int>(a.M);
   gp.N = static_cast<int>(a.N);
   gp.K = static_cast<int>(a.K);
   gp.y = a.y;
   gp.scales = nullptr;
-  const dim3 grid(static_cast<unsigned>(2 * pairs_n), static_cast<unsigned>((a.M + bt - 1) / bt));
+  GemmPairTiles tl;
+  tl.tiles_n = static_cast<int>(pairs_n);
+  tl.tiles_m = static_cast<int>((a.M + bt - 1) / bt);
+  const int64_t ntiles = pairs_n * tl.tiles_m;
+  const dim3 grid(static_cast<unsigned>(2 * std::min<int64_t>(ntiles, std::max(1, d->sm_count / 2))));
 #define TB_GI8_LAUNCH(BT, F)                                                                                  \
   {                                                                                                           \
     auto k = gemm_pair_kernel<BT, int32_t, F, true>;                                                          \
     if (allow_smem(k, d) != TB_OK) return TB_ERR_CUDA;                                                        \
     return launch_pdl(k, grid, dim3(kGpThreads), static_cast<size_t>(gp_smem_bytes(BT, F, true)), a.st, tm_x, \
-                      tm_w, tm_y, gp, tma_y);                                                                 \
+                      tm_w, gp, tl);                                                                          \
   }
   if (bt == 128) {
     if (one_bit) TB_GI8_LAUNCH(128, 2)
