@@ -480,10 +480,21 @@ def run_prefill(args, dev, stream, tb, inputs, world=1, integer=False):
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": round(peak, 1),
                          "unit": "TFLOP/s" if not integer else "TOP/s", "frac": round(tflops / peak, 4),
                          "peak_source": kind,
+                         "frac_of_sustained": _sustained_frac(tflops, integer),
                          "dtype": "s8 x s8 -> s32 (kind::i8)" if integer else "fp16 x fp16 -> fp32 (kind::f16)",
                          "kernel": "gemm_pair_kernel (CTA pairs, cta_group::2, A = unpacked weights in TMEM)"},
             "clocks": clocks,
             "kernel_path": tb.tb_ternary_linear_path(xt, "2bit", m, n, k, not integer, True)}
+
+
+def _sustained_frac(tflops, integer):
+    """The same figure against the sustained (seconds-long, power-capped) bf16 measurement, for context."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            sus = float(json.load(f)["bf16_tflops_sustained"])
+    except (OSError, KeyError, ValueError):
+        return None
+    return round(tflops / (sus * (2.0 if integer else 1.0)), 4)
 
 
 def _tensor_peak():
