@@ -69,6 +69,18 @@ def test_int8_gemm_bitexact(case, fmt):
     assert np.array_equal(got, orc.linear_int(x, codes))
 
 
+@pytest.mark.parametrize("fmt", ["2bit", "1bit"])
+def test_int8_gemm_several_tiles_per_cluster(fmt):
+    """94 pair tiles (more than the clusters), ragged M and N, and K = 640: the
+    last stage holds 128 of its 256 codes (the copies read zeros past K)."""
+    rng = np.random.default_rng(70)
+    m, n, k = 300, 12000, 640
+    codes = _codes(rng, n, k, fmt)
+    x = rng.integers(-128, 128, (m, k)).astype(np.int8)
+    got = _run(fmt, codes, x, path=GEMM)
+    assert np.array_equal(got, orc.linear_int(x, codes))
+
+
 def test_int8_extreme_values():
     """Every activation -128 or 127 and every code +-1: the largest sums."""
     rng = np.random.default_rng(66)

@@ -293,6 +293,22 @@ def test_gemm_prefill_full_size_sampled_rows():
     assert np.isfinite(y).all()
 
 
+@pytest.mark.parametrize("fmt", ["2bit", "1bit"])
+@pytest.mark.parametrize("m,n,k", [(777, 9000, 1024),     # 4 x 36 tiles, ragged M and N (last CTA pair half empty)
+                                   (100, 40000, 1024)])   # 128-token tiles, 157 of them
+def test_gemm_several_tiles_per_cluster(fmt, m, n, k):
+    """More pair tiles than clusters: each cluster walks two or three tiles
+    (the read-out of one tile overlapping the next tile's first stages), with
+    ragged token and row tiles; the whole output against the oracle, in fp32
+    and bf16, and two calls give identical bits."""
+    p0 = 0.33 if fmt == "2bit" else 0.0
+    prob, ref = _problem(29, m, n, k, p0, fmt)
+    y = prob.linear(GEMM)
+    _check(y, ref, prob.p)
+    assert np.array_equal(y, prob.linear(GEMM))
+    _check(prob.linear(GEMM, yt=tb.TB_BF16), ref, prob.p)
+
+
 def test_gemm_invalid_bytes_no_fault():
     prob, _ = _problem(20, 5, 256, 1024, 1 / 3, "2bit")
     y = prob.linear(GEMM, packed=torch.full_like(prob.packed, 0xFF))
