@@ -81,6 +81,19 @@ def test_int8_gemm_several_tiles_per_cluster(fmt):
     assert np.array_equal(got, orc.linear_int(x, codes))
 
 
+@pytest.mark.parametrize("fmt", ["2bit", "1bit"])
+def test_int8_long_k_with_and_without_workspace(fmt):
+    """Few tiles and long K (17408: 68 stages of 256 codes), with and without a
+    workspace (integer mode needs none for 2-bit and 1-bit): both exact."""
+    rng = np.random.default_rng(71)
+    m, n, k = 40, 700, 17408
+    codes = _codes(rng, n, k, fmt)
+    x = rng.integers(-128, 128, (m, k)).astype(np.int8)
+    ref = orc.linear_int(x, codes)
+    assert np.array_equal(_run(fmt, codes, x, with_ws=True, path=GEMM), ref)
+    assert np.array_equal(_run(fmt, codes, x, with_ws=False, path=GEMM), ref)
+
+
 def test_int8_extreme_values():
     """Every activation -128 or 127 and every code +-1: the largest sums."""
     rng = np.random.default_rng(66)

@@ -309,6 +309,17 @@ def test_gemm_several_tiles_per_cluster(fmt, m, n, k):
     _check(prob.linear(GEMM, yt=tb.TB_BF16), ref, prob.p)
 
 
+def test_gemm_few_tiles_long_k_deterministic():
+    """Few tiles (4 pair tiles) and long K (17408, 136 stages a tile): repeated
+    calls give identical bits, in fp32 and bf16."""
+    prob, ref = _problem(31, 64, 1000, 17408, 0.5, "2bit", "lognormal", 0.0)
+    y = prob.linear(GEMM)
+    _check(y, ref, prob.p)
+    for _ in range(3):
+        assert np.array_equal(y, prob.linear(GEMM))
+    _check(prob.linear(GEMM, yt=tb.TB_BF16), ref, prob.p)
+
+
 def test_gemm_invalid_bytes_no_fault():
     prob, _ = _problem(20, 5, 256, 1024, 1 / 3, "2bit")
     y = prob.linear(GEMM, packed=torch.full_like(prob.packed, 0xFF))
